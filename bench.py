@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark of the per-group low-bit quantized linear hot path on B200.
+
+One step = the whole hot path over the FLUX-like DiT linears (4-bit, group 128, rank-32
+bf16 branch, bias, M = 4096 tokens): for each of W 3072x3072, 12288x3072 and 3072x12288,
+quantize + pack the residual weight (wq_quantize_pack), then run the fused dequant-GEMM
+y = x deq(R)^T + (x L1) L2 + bias (wq_linear).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). `value` is the dequant-GEMM throughput of the whole step
+(algorithmic GEMM FLOPs of all ranks / device time of the step, max over ranks), in TFLOP/s.
+Multi-GPU runs are independent replicas (the path has no exchange step): weak scaling.
+`--impl reference` times the CPU oracle (the only baseline for this method) on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dequant-GEMM TFLOP/s & weight GB/s (% roofline); quantize+pack Gparam/s"
+WORKLOAD = ("FLUX-like DiT linears W 3072x3072, 12288x3072, 3072x12288; M=4096 tokens; "
+            "4-bit per-group(128); rank-32 bf16 low-rank branch; bias; step = quantize+pack + dequant-GEMM")
+BITS, RANK, M_TOKENS = 4, 32, 4096
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_flops(N, K, M, rank):
+    return 2.0 * M * N * K + 2.0 * M * rank * (K + N)
+
+
+def weight_bytes(N, K, bits):
+    return N * K * bits / 8 + N * K / 128 * 4
+
+
+def dist_info():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML from a background thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.error = str(e)
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "nvml")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- workload
+
+def make_workload(device):
+    """Seeded synthetic FLUX-like linears, resident on `device`, plus their host copies."""
+    import numpy as np
+    import torch
+    from bit_weight_quantization_wq_b200 import synth
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+    lins = synth.flux_linears(M=M_TOKENS, rank=RANK)
+    out = []
+    for lin in lins:
+        N, K = lin["N"], lin["K"]
+        d = dict(N=N, K=K, host=lin,
+                 R=dev(lin["R"]), x=dev(lin["x"]), L1=dev(lin["L1"]), L2=dev(lin["L2"]), bias=dev(lin["bias"]),
+                 packed=torch.empty((N, K * BITS // 8), dtype=torch.uint8, device=device),
+                 scales=torch.empty((N, K // 128), dtype=torch.float32, device=device),
+                 y=torch.empty((M_TOKENS, N), dtype=torch.bfloat16, device=device))
+        out.append(d)
+    return out
+
+
+def run_step(wq, lins, ws, events=None):
+    for i, d in enumerate(lins):
+        if events is not None:
+            events[i][0].record()
+        wq.wq_quantize_pack(d["R"], BITS, packed=d["packed"], scales=d["scales"])
+        if events is not None:
+            events[i][1].record()
+        wq.wq_linear(d["x"], d["packed"], d["scales"], BITS, d["N"], L1=d["L1"], L2=d["L2"],
+                     bias=d["bias"], y=d["y"], workspace=ws)
+        if events is not None:
+            events[i][2].record()
+
+
+# ----------------------------------------------------------------------------- oracle legs
+
+def oracle_sample(lins_host, rows_per_linear: int, pack_rows: int):
+    """Run the CPU oracle on a bounded sample: quantize + pack `pack_rows` weight rows of each
+    residual, dequantize those rows, and evaluate the fp64 linear for `rows_per_linear` token
+    rows against them (scaled to the full output width). Returns (flops, params, seconds)."""
+    import numpy as np
+    import oracle
+    flops = params = 0.0
+    t0 = time.perf_counter()
+    for i, lin in enumerate(lins_host):
+        N, K = lin["N"], lin["K"]
+        n = min(pack_rows, N)
+        codes, scales = oracle.quantize(lin["R"][:n], BITS)
+        oracle.pack(codes, BITS)
+        deq = oracle.dequant(codes, scales, BITS)
+        rows = np.arange(rows_per_linear, dtype=np.int64) + 17 * i
+        oracle.linear_rows(lin["x"], deq, lin["L1"], lin["L2"][:, :n], lin["bias"][:n], rows)
+        flops += gemm_flops(n, K, rows_per_linear, RANK)
+        params += n * K
+    return flops, params, time.perf_counter() - t0
+
+
+def cpu_baseline(lins_host, budget_s: float = 12.0):
+    import oracle
+    f, p, t = oracle_sample(lins_host, 4, 1024)          # calibration
+    scale = max(1.0, budget_s / max(t, 1e-3))
+    rows = max(4, min(512, int(4 * scale)))
+    prow = max(256, min(3072, int(1024 * scale)))
+    f, p, t = oracle_sample(lins_host, rows, prow)
+    return {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"C oracle (fp32 quantize+pack, fp64 linear with the rank-32 branch) on {prow} weight rows "
+                       f"of each of the 3 residuals x {rows} token rows: {f / 1e9:.2f} GFLOP in {t:.1f} s; "
+                       f"oracle pack rate {p / t / 1e9:.4f} Gparam/s (pack+dequant+linear wall time)")}
+
+
+def reference_arm(args):
+    """--impl reference: the CPU oracle timed on bounded samples of the workload."""
+    world, rank, _ = dist_info()
+    if rank != 0:
+        return 0
+    import oracle
+    from bit_weight_quantization_wq_b200 import synth
+    lins_host = synth.flux_linears(M=M_TOKENS, rank=RANK)
+    steps, warmup = args.steps, args.warmup
+    f, p, t = oracle_sample(lins_host, 2, 256)
+    per_step = max(1.0, min(20.0, 90.0 / max(1, steps + warmup)))
+    scale = max(1.0, per_step / max(t, 1e-3))
+    rows, prow = max(2, min(256, int(2 * scale))), max(128, min(3072, int(256 * scale)))
+    for _ in range(warmup):
+        oracle_sample(lins_host, rows, prow)
+    tot_f = tot_t = 0.0
+    for _ in range(steps):
+        f, p, t = oracle_sample(lins_host, rows, prow)
+        tot_f += f
+        tot_t += t
+    value = tot_f / tot_t / 1e12 if tot_t > 0 else 0.0
+    sample = (f"per step: C oracle on {prow} weight rows of each of the 3 residuals x {rows} token rows "
+              f"({tot_f / max(steps, 1) / 1e9:.2f} GFLOP)")
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": steps,
+            "warmup": warmup, "ms_per_step": 1e3 * tot_t / max(steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": sample}, "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "kind": "oracle", "cores": oracle.num_threads(),
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- main arm
+
+def main_arm(args):
+    import torch
+    import bit_weight_quantization_wq_b200 as wq
+    from bit_weight_quantization_wq_b200 import build as wq_build
+
+    world, rank, local = dist_info()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    if rank == 0:
+        wq_build.build()
+    barrier(world, device)
+    wq.lib()
+
+    lins = make_workload(device)
+    ws = torch.empty(max(wq.wq_linear_workspace_bytes(M_TOKENS, d["N"], d["K"], BITS, RANK) for d in lins),
+                     dtype=torch.uint8, device=device)
+    step_flops = sum(gemm_flops(d["N"], d["K"], M_TOKENS, RANK) for d in lins)
+    step_params = sum(d["N"] * d["K"] for d in lins)
+    step_wbytes = sum(weight_bytes(d["N"], d["K"], BITS) for d in lins)
+
+    for _ in range(args.warmup):
+        run_step(wq, lins, ws)
+    torch.cuda.synchronize()
+    if wq.wq_device_status() != 0:
+        raise RuntimeError("device status not clean after warm-up")
+
+    # ---------------------------------------------------------------- timed region
+    K = args.steps
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in lins] for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    torch.cuda.synchronize()
+    launches0 = wq.wq_launch_count()
+    with ClockSampler(device.index) as clocks:
+        start.record()
+        for k in range(K):
+            run_step(wq, lins, ws, ev[k])
+        stop.record()
+        torch.cuda.synchronize()
+    launches = wq.wq_launch_count() - launches0
+    barrier(world, device)
+    step_ms = start.elapsed_time(stop) / K
+    step_ms = max_over_ranks(step_ms, world, device)
+    pack_ms = sum(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(K) for i in range(len(lins))) / K
+    lin_ms = sum(ev[k][i][1].elapsed_time(ev[k][i][2]) for k in range(K) for i in range(len(lins))) / K
+    if wq.wq_device_status() != 0:
+        raise RuntimeError("device status not clean after the timed region")
+
+    peaks, peak_src = load_peaks()
+    lin_tflops = step_flops / (lin_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": lin_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": lin_tflops / peaks["bf16_tflops"], "traffic": None,
+                "kernel": "wq_linear (lowrank_prepass_kernel + tc_linear_kernel<4>), mean over the 3 shapes",
+                "peak_source": f"{peak_src} bf16 dense (burst)"}
+
+    # ---------------------------------------------------------------- e2e through host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_leg(wq, lins, ws, args, device, world, step_flops)
+
+    value = step_flops * world / (step_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_tokens": M_TOKENS * world, "bits": BITS, "group": 128,
+                   "rank": RANK, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2: a step reads ~320 MB of distinct inputs, so each kernel's "
+                         "operands were evicted by the rest of the step before it runs again"},
+        "roofline": roofline,
+        "breakdown": {
+            "linear_ms_per_step": lin_ms, "pack_ms_per_step": pack_ms,
+            "linear_tflops": lin_tflops,
+            "linear_weight_gbs": step_wbytes / (lin_ms * 1e-3) / 1e9,
+            "pack_gparams": step_params / (pack_ms * 1e-3) / 1e9,
+            "pack_gbs": (2 * step_params + step_wbytes) / (pack_ms * 1e-3) / 1e9,
+            "pack_hbm_frac": (2 * step_params + step_wbytes) / (pack_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        },
+        "clocks": clocks.summary(),
+        "gpu_launches": launches,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline([d["host"] for d in lins], budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def e2e_leg(wq, lins, ws, args, device, world, step_flops):
+    """Same metric through the public API with HOST buffers: every step copies its inputs
+    from pinned host memory and reads the outputs back."""
+    import numpy as np
+    import torch
+    host_in, host_out = [], []
+    for d in lins:
+        h = d["host"]
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+        host_in.append({k: pin(h[k]) for k in ("R", "x", "L1", "L2", "bias")})
+        host_out.append(torch.empty((M_TOKENS, d["N"]), dtype=torch.bfloat16).pin_memory())
+    h2d = sum(t.numel() * 2 for hi in host_in for t in hi.values())
+    d2h = sum(t.numel() * 2 for t in host_out)
+
+    def step():
+        for d, hi, ho in zip(lins, host_in, host_out):
+            for k, t in hi.items():
+                d[k].copy_(t, non_blocking=True)
+            wq.wq_quantize_pack(d["R"], BITS, packed=d["packed"], scales=d["scales"])
+            wq.wq_linear(d["x"], d["packed"], d["scales"], BITS, d["N"], L1=d["L1"], L2=d["L2"],
+                         bias=d["bias"], y=d["y"], workspace=ws)
+            ho.copy_(d["y"], non_blocking=True)
+
+    steps = max(3, min(args.steps, 20))
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps):
+        step()
+    stop.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(stop) / steps, world, device)
+    return {"value": step_flops * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    return ap.parse_args(argv)
+
+
+def main(argv=None):
+    args = parse(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return reference_arm(args)
+    return main_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

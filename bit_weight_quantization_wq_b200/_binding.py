@@ -1,0 +1,197 @@
+"""ctypes binding of libwq.so (include/wq.h). Argument marshalling only.
+
+Every call takes torch CUDA tensors and passes their device pointers, sizes and the
+current torch stream to the C ABI; all computation runs in the library's kernels. There is
+no fallback: if ``libwq.so`` is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libwq.so")
+
+# wq_status codes (include/wq.h)
+WQ_OK = 0
+WQ_ERR_INVALID_ARG = 1
+WQ_ERR_UNSUPPORTED_BITS = 2
+WQ_ERR_UNSUPPORTED_GROUP = 3
+WQ_ERR_MISALIGNED = 4
+WQ_ERR_CUDA = 5
+WQ_ERR_TIMEOUT = 6
+WQ_ERR_WORKSPACE = 7
+WQ_ERR_UNSUPPORTED_DEVICE = 8
+
+PATHS = {"auto": 0, "small_m": 1, "tensor": 2}
+
+# exported C symbols, as declared in include/wq.h
+SYMBOLS = (
+    "wq_version", "wq_packed_bytes", "wq_scales_count", "wq_quantize_pack",
+    "wq_linear_workspace_bytes", "wq_linear", "wq_linear_ex", "wq_device_status",
+    "wq_selftest_bounded_wait", "wq_status_string", "wq_last_error", "wq_launch_count",
+)
+
+
+class WQError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        msg = f"{where}: {status_string(status)} (status {status})"
+        if detail:
+            msg += f": {detail}"
+        super().__init__(msg)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libwq.so from the package directory. Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libwq.so not found at {LIB_PATH}; build it with "
+                "`python -m bit_weight_quantization_wq_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        i64, i32, sz, p = ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+        L.wq_version.argtypes, L.wq_version.restype = [], i32
+        L.wq_packed_bytes.argtypes, L.wq_packed_bytes.restype = [i64, i64, i32], sz
+        L.wq_scales_count.argtypes, L.wq_scales_count.restype = [i64, i64, i32], i64
+        L.wq_quantize_pack.argtypes = [p, i64, i64, i32, i32, p, p, p]
+        L.wq_quantize_pack.restype = i32
+        L.wq_linear_workspace_bytes.argtypes = [i64, i64, i64, i32, i32]
+        L.wq_linear_workspace_bytes.restype = sz
+        L.wq_linear.argtypes = [p, i64, i64, p, p, i32, i32, i64, p, p, i32, p, p, p, sz, p]
+        L.wq_linear.restype = i32
+        L.wq_linear_ex.argtypes = [p, i64, i64, p, p, i32, i32, i64, p, p, i32, p, p, p, sz, i32, p]
+        L.wq_linear_ex.restype = i32
+        L.wq_device_status.argtypes, L.wq_device_status.restype = [p, i32], i32
+        L.wq_selftest_bounded_wait.argtypes = [ctypes.c_uint32, p]
+        L.wq_selftest_bounded_wait.restype = i32
+        L.wq_status_string.argtypes, L.wq_status_string.restype = [i32], ctypes.c_char_p
+        L.wq_last_error.argtypes, L.wq_last_error.restype = [], ctypes.c_char_p
+        L.wq_launch_count.argtypes, L.wq_launch_count.restype = [], ctypes.c_uint64
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().wq_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != WQ_OK:
+        raise WQError(status, where, lib().wq_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t, name, dtype, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+# ----------------------------------------------------------------------------- API
+
+def wq_version() -> int:
+    return int(lib().wq_version())
+
+
+def wq_packed_bytes(N: int, K: int, bits: int) -> int:
+    return int(lib().wq_packed_bytes(N, K, bits))
+
+
+def wq_scales_count(N: int, K: int, group: int = 128) -> int:
+    return int(lib().wq_scales_count(N, K, group))
+
+
+def wq_linear_workspace_bytes(M: int, N: int, K: int, bits: int, rank: int = 0) -> int:
+    return int(lib().wq_linear_workspace_bytes(M, N, K, bits, rank))
+
+
+def wq_quantize_pack(W, bits: int, group: int = 128, packed=None, scales=None, stream=None):
+    """Quantize + pack an (N, K) bf16 weight. Returns (packed uint8 (N, K*bits/8), scales f32 (N, K/group))."""
+    import torch
+    _dev(W, "W", torch.bfloat16)
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D (N, K)")
+    N, K = W.shape
+    if packed is None:
+        packed = torch.empty((N, K * bits // 8), dtype=torch.uint8, device=W.device)
+    if scales is None:
+        scales = torch.empty((N, max(K // group, 0)), dtype=torch.float32, device=W.device)
+    _dev(packed, "packed", torch.uint8)
+    _dev(scales, "scales", torch.float32)
+    st = lib().wq_quantize_pack(_ptr(W), N, K, bits, group, _ptr(packed), _ptr(scales), _stream(stream))
+    _check(st, "wq_quantize_pack")
+    return packed, scales
+
+
+def wq_linear(x, packed, scales, bits: int, N: int, L1=None, L2=None, bias=None, y=None,
+              workspace=None, group: int = 128, path: str = "auto", stream=None):
+    """y = x dequant(packed, scales)^T + (x L1) L2 + bias, bf16 (M, N)."""
+    import torch
+    _dev(x, "x", torch.bfloat16)
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D (M, K)")
+    M, K = x.shape
+    _dev(packed, "packed", torch.uint8)
+    _dev(scales, "scales", torch.float32)
+    rank = 0
+    if L1 is not None or L2 is not None:
+        if L1 is None or L2 is None:
+            raise ValueError("L1 and L2 go together")
+        _dev(L1, "L1", torch.bfloat16)
+        rank = L1.shape[1]
+        _dev(L2, "L2", torch.bfloat16, (rank, N))
+    if bias is not None:
+        _dev(bias, "bias", torch.bfloat16, (N,))
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _dev(y, "y", torch.bfloat16, (M, N))
+    need = wq_linear_workspace_bytes(M, N, K, bits, rank)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().wq_linear_ex(_ptr(x), M, K, _ptr(packed), _ptr(scales), bits, group, N,
+                            _ptr(L1), _ptr(L2), rank, _ptr(bias), _ptr(y), _ptr(workspace),
+                            ws_bytes, PATHS[path], _stream(stream))
+    _check(st, "wq_linear")
+    return y
+
+
+def wq_device_status(stream=None, clear: bool = True) -> int:
+    """Synchronize and return the device-side status (raises on WQ_ERR_CUDA)."""
+    st = lib().wq_device_status(_stream(stream), 1 if clear else 0)
+    if st == WQ_ERR_CUDA:
+        _check(st, "wq_device_status")
+    return st
+
+
+def wq_launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(lib().wq_launch_count())
+
+
+def wq_selftest_bounded_wait(timeout_us: int, stream=None) -> int:
+    return int(lib().wq_selftest_bounded_wait(timeout_us, _stream(stream)))

