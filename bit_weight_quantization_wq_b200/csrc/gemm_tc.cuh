@@ -1,30 +1,36 @@
 // gemm_tc.cuh -- large-M fused dequant-GEMM on the 5th-generation tensor cores (KL).
 //
-//   y = x * dequant(W)^T + (x L1) L2 + bias
+//   y = x * dequant(W)^T + (x L1) L2 + bias,   dequant(code) = (code - 2^(b-1)) * step
 //
 // The Per-group(128) article dequantizes each block's weights on the GPU (sec. 3.4) and
 // then runs a bf16 matmul, noting it has no low-bit matmul kernel (sec. 5.3, 5.4); the
 // SVDQuant article adds a 16-bit low-rank branch computed next to the quantized residual
-// ("Technical principles", "Engineering highlights"). Here the dequantization happens in
-// registers inside the GEMM: the bf16 weight is never written to global memory.
+// ("Technical principles", "Engineering highlights"). Here the weight is never
+// dequantized to memory, and never rounded: the tensor cores multiply the exact integer
+// codes q = code - 2^(b-1) (exact in bf16) by x, one 128-wide group at a time, and each
+// group's fp32 partial product is scaled by its fp32 step and added to the result:
 //
-// One persistent CTA per SM walks 256 x 256 output tiles (256 tokens x 256 weight rows).
+//   y[m][n] = sum_g step[n][g] * ( sum_{k in g} q[n][k] x[m][k] )  (+ low-rank, + bias)
+//
+// Orientation: D = W_q x^T, so TMEM lanes are weight rows and columns are tokens; the
+// per-group step is then one scalar per lane.
+// One persistent CTA per SM walks 128 x 128 tiles (128 weight rows x 128 tokens).
+// TMEM (512 columns): T0, T1 = per-group partials (double-buffered, 128 columns each),
+// R = running sum (128), A = 4 stages of codes (32 columns = 64 k each).
 // Warp roles (384 threads):
-//   warp 0     TMA producer of x tiles (256 tokens x 64 k bf16, 128B-swizzled, 32 KB/stage)
-//   warp 1     TMEM allocator and the single MMA-issuing thread: per 64-k stage, 4 k-steps of
-//              two tcgen05.mma M=128 N=256 K=16 (one per token half) into two fp32 TMEM
-//              accumulators (2 x 256 columns = all 512)
-//   warp 2     TMA producer of packed-weight tiles (256 rows x one 128-code group)
-//   warps 4-11 dequantizers, one weight row per thread: unpack 8 codes at a time from the
-//              packed tile, dequantize in fp32 ((code - 2^(b-1)) * step as one FMA on the
-//              exponent-trick value 1 + code/128), round to bf16 and store the 128B-swizzled
-//              K-major B operand the MMA reads; after the k loop they run the epilogue
-//              (tcgen05.ld, + bias, round to bf16, store y).
-// Low-rank branch: y = [x, t] [deq(W)^T ; L2] with t = bf16(x L1) (M x rank, computed by
-// lowrank_prepass_kernel), so it is one more k stage into the same accumulators.
+//   warp 0      TMA producer of x tiles (128 tokens x 64 k bf16, 128B swizzle, 16 KB/stage)
+//   warp 1      TMEM allocator; one thread issues tcgen05.mma (A = codes from TMEM,
+//               B = x from shared memory, M=128 N=128 K=16) into T
+//   warps 4-7   unpack: one weight row per thread; packed bytes come from global memory
+//               straight into registers (two groups ahead), become bf16 pairs of exact q
+//               and are written to the A stage with tcgen05.st
+//   warps 8-11  promotion: R += step * T per group (fp32, two lanes per instruction), then the
+//               epilogue (+ bias, round once to bf16, store y)
+// Low-rank branch: one more unit per tile with A = L2^T (bf16 from global) and B = the
+// t = bf16(x L1) tile, promoted with scale 1 into the same R.
 //
-// Every wait is bounded (see common.cuh). On a timeout the roles stop, the producers wait
-// (bounded) for their copies in flight, the MMA thread for its MMAs, and TMEM is freed.
+// Every wait is bounded (see common.cuh). On a timeout the roles stop, the producer waits
+// (bounded) for its copies in flight, the MMA thread for its MMAs, and TMEM is freed.
 #pragma once
 
 #include <cuda.h>
@@ -34,34 +40,30 @@
 
 namespace wq {
 
-constexpr int kTcBM = 256;
-constexpr int kTcBN = 256;
-constexpr int kTcBK = 64;
-constexpr int kTcStagesA = 3;
-constexpr int kTcStagesB = 2;
-constexpr int kTcStagesP = 2;
+constexpr int kTcBW = 128;                // weight rows per tile (MMA M)
+constexpr int kTcBT = 128;                // tokens per tile (MMA N)
+constexpr int kTcBK = 64;                 // k per x stage / A stage
+constexpr int kTcStagesX = 6;
+constexpr int kTcStagesA = 4;
 constexpr int kTcThreads = 384;
-constexpr int kTcFirstDequantWarp = 4;
-constexpr int kTcDequantWarps = 8;
+constexpr int kTcUnpackWarp0 = 4;
+constexpr int kTcPromoteWarp0 = 8;
 constexpr uint32_t kTcTmemCols = 512;
+constexpr uint32_t kTmemT0 = 0, kTmemR = 256, kTmemA = 384;
 constexpr int kTStride = 64;              // row stride (elements) of the low-rank t buffer
 
-template <int BITS>
 struct TcLayout {
-    static constexpr uint32_t kABytes = kTcBM * kTcBK * 2;
-    static constexpr uint32_t kBBytes = kTcBN * kTcBK * 2;
-    static constexpr uint32_t kPBytes = kTcBN * 16 * BITS;
-    static constexpr uint32_t kOffA = 0;
-    static constexpr uint32_t kOffB = kOffA + kTcStagesA * kABytes;
-    static constexpr uint32_t kOffP = kOffB + kTcStagesB * kBBytes;
-    static constexpr uint32_t kOffBar = kOffP + kTcStagesP * kPBytes;
-    static constexpr uint32_t kNumBars = 2 * kTcStagesA + 2 * kTcStagesB + 2 * kTcStagesP + 3;
+    static constexpr uint32_t kXBytes = kTcBT * kTcBK * 2;          // 16 KB
+    static constexpr uint32_t kOffX = 0;
+    static constexpr uint32_t kOffBar = kOffX + kTcStagesX * kXBytes;
+    static constexpr uint32_t kNumBars = 2 * kTcStagesX + 2 * kTcStagesA + 4 + 1;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kBytes = kOffMisc + 16;
-    static constexpr uint32_t kAlloc = kBytes + 1024;     // slack to align the base to 1024 B
+    static constexpr uint32_t kAlloc = kBytes + 1024;               // slack to align the base to 1024 B
 };
 
 struct TcParams {
+    const uint8_t *packed;    // N x K*bits/8
     const float *scales;      // N x K/128
     const uint16_t *L2;       // rank x N bf16 or null
     const uint16_t *bias;     // N bf16 or null
@@ -96,16 +98,62 @@ __device__ __forceinline__ void tc_block_be(const uint32_t (&w)[NW], uint32_t &l
     }
 }
 
-// Code I of a big-endian block as the fp32 value 1 + code/128 (code placed at mantissa bit 16).
-template <int BITS, int I>
-__device__ __forceinline__ float tc_code_f32(uint32_t lo, uint32_t hi) {
-    constexpr int sh = BITS * (7 - I);
-    constexpr uint32_t m = ((1u << BITS) - 1u) << 16;
-    uint32_t v;
-    if constexpr (sh >= 48) v = hi >> (sh - 48);
-    else if constexpr (sh >= 16) v = __funnelshift_r(lo, hi, sh - 16);
-    else v = lo << (16 - sh);
-    return __uint_as_float((v & m) | 0x3F800000u);
+// PTX prmt in its default mode: selector nibble bits 2:0 pick one of the 8 source bytes and
+// bit 3 replaces it by copies of that byte's sign bit (zero for bytes below 0x80). The CUDA
+// __byte_perm intrinsic ignores bit 3, hence the inline form.
+__device__ __forceinline__ uint32_t prmt_sx(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// 32 bf16x2 words of exact q = code - 2^(b-1), in natural k order (word i = k 2i, 2i+1),
+// for codes [64 h, 64 h + 64) of a group held as 4*b little-endian words.
+template <int BITS, int H, int NW>
+__device__ __forceinline__ void unpack_half(const uint32_t (&w)[NW], uint32_t (&out)[32]) {
+    constexpr uint32_t kOff = 0x43004300u;                          // bf16 128 in each half
+    const __nv_bfloat162 corr = __floats2bfloat162_rn(128.0f + (1 << (BITS - 1)), 128.0f + (1 << (BITS - 1)));
+    if constexpr (BITS == 4) {
+        // byte j of a word = (code 2j << 4) | code 2j+1
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t v = w[8 * H + i];
+            const uint32_t hiN = (v >> 4) & 0x0F0F0F0Fu, loN = v & 0x0F0F0F0Fu;
+            // (hi nibble of byte j) | (lo nibble of byte j) << 16; the sign-replicating
+            // selector nibbles (8 + byte) give the zero high bytes
+            const uint32_t p0 = prmt_sx(hiN, loN, 0xC480u) + kOff;
+            const uint32_t p1 = prmt_sx(hiN, loN, 0xD591u) + kOff;
+            const uint32_t p2 = prmt_sx(hiN, loN, 0xE6A2u) + kOff;
+            const uint32_t p3 = prmt_sx(hiN, loN, 0xF7B3u) + kOff;
+            const uint32_t pp[4] = {p0, p1, p2, p3};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                __nv_bfloat162 t = *reinterpret_cast<const __nv_bfloat162 *>(&pp[j]);
+                t = __hsub2(t, corr);
+                out[4 * i + j] = *reinterpret_cast<uint32_t *>(&t);
+            }
+        }
+    } else {
+        constexpr uint32_t m = (1u << BITS) - 1u;
+        static_for<8>([&](auto bb) {
+            constexpr int blk = decltype(bb)::value;
+            uint32_t lo, hi;
+            tc_block_be<BITS, 8 * H + blk>(w, lo, hi);
+            static_for<4>([&](auto pp) {
+                constexpr int pr = decltype(pp)::value;
+                constexpr int sh = 2 * BITS * (3 - pr);
+                uint32_t G;
+                if constexpr (sh >= 32) G = hi >> (sh - 32);
+                else if constexpr (sh == 0) G = lo;
+                else G = __funnelshift_r(lo, hi, sh);
+                // G bits [0,b) = code 2pr+1, [b,2b) = code 2pr: low half <- G >> b, high half <- G
+                uint32_t r = (__byte_perm(G >> BITS, G, 0x5410u) & (m | (m << 16))) | kOff;
+                __nv_bfloat162 t = *reinterpret_cast<const __nv_bfloat162 *>(&r);
+                t = __hsub2(t, corr);
+                out[4 * blk + pr] = *reinterpret_cast<uint32_t *>(&t);
+            });
+        });
+    }
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -139,30 +187,37 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 template <int BITS>
+__device__ __forceinline__ void load_group(const uint8_t *src, bool ok, uint32_t (&w)[4 * BITS + 1]) {
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) {
+        const uint4 v = ok ? __ldg(reinterpret_cast<const uint4 *>(src) + i) : make_uint4(0, 0, 0, 0);
+        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+    }
+    w[4 * BITS] = 0;
+}
+
+template <int BITS>
 __global__ void __launch_bounds__(kTcThreads, 1)
-tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap p_map,
-                 const __grid_constant__ CUtensorMap t_map, const TcParams p) {
-    using L = TcLayout<BITS>;
-    constexpr int SA = kTcStagesA, SB = kTcStagesB, SP = kTcStagesP;
-    constexpr int kHalf = 1 << (BITS - 1);
+tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap t_map,
+                 const TcParams p) {
+    using L = TcLayout;
+    constexpr int SX = kTcStagesX, SA = kTcStagesA;
+    constexpr int NWG = 4 * BITS + 1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
-    uint64_t *a_full = bars, *a_empty = a_full + SA;
-    uint64_t *b_full = a_empty + SA, *b_empty = b_full + SB;
-    uint64_t *p_full = b_empty + SB, *p_empty = p_full + SP;
-    uint64_t *acc_full = p_empty + SP, *acc_empty = acc_full + 1, *drain = acc_empty + 1;
+    uint64_t *x_full = bars, *x_empty = x_full + SX;
+    uint64_t *a_full = x_empty + SX, *a_empty = a_full + SA;
+    uint64_t *t_full = a_empty + SA, *t_empty = t_full + 2, *drain = t_empty + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < SA; ++i) { mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 1); }
-        for (int i = 0; i < SB; ++i) { mbar_init(&b_full[i], kTcDequantWarps); mbar_init(&b_empty[i], 1); }
-        for (int i = 0; i < SP; ++i) { mbar_init(&p_full[i], 1); mbar_init(&p_empty[i], kTcDequantWarps); }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, kTcDequantWarps);
+        for (int i = 0; i < SX; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
+        for (int i = 0; i < SA; ++i) { mbar_init(&a_full[i], 4); mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&t_full[i], 1); mbar_init(&t_empty[i], 4); }
         mbar_init(drain, 1);
         *abort = 0;
         fence_barrier_init();
@@ -176,85 +231,66 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    const int KBm = (int)(p.K / kTcBK);              // k stages of the quantized weight
-    const int KB = KBm + (p.rank > 0 ? 1 : 0);       // + the low-rank stage
     const int G = (int)(p.K / 128);
+    const int U = G + (p.rank > 0 ? 1 : 0);          // units per tile: groups (+ low-rank)
     const int tiles = p.tiles_m * p.tiles_n;
 
     if (warp == 0 && lane == 0) {
         // ---------------------------------------------------------- x / t producer
         tma_prefetch_desc(&x_map);
         tma_prefetch_desc(&t_map);
-        int armed[SA];
-        for (int i = 0; i < SA; ++i) armed[i] = -1;
+        int armed[SX];
+        for (int i = 0; i < SX; ++i) armed[i] = -1;
         uint32_t s = 0, ph = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int mt = tile % p.tiles_m;
-            for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(&a_empty[s], ph ^ 1, abort)) goto a_done;
-                mbar_arrive_expect_tx(&a_full[s], L::kABytes);
-                armed[s] = (int)ph;
-                uint8_t *dst = smem + L::kOffA + s * L::kABytes;
-                if (kb < KBm) tma_load_2d(dst, &x_map, &a_full[s], kb * kTcBK, mt * kTcBM);
-                else tma_load_2d(dst, &t_map, &a_full[s], 0, mt * kTcBM);
-                if (++s == SA) { s = 0; ph ^= 1; }
+            for (int u = 0; u < U; ++u) {
+                const int nst = (u < G) ? 2 : 1;
+                for (int st = 0; st < nst; ++st) {
+                    if (!mbar_wait(&x_empty[s], ph ^ 1, abort)) goto x_done;
+                    mbar_arrive_expect_tx(&x_full[s], L::kXBytes);
+                    armed[s] = (int)ph;
+                    uint8_t *dst = smem + L::kOffX + s * L::kXBytes;
+                    if (u < G) tma_load_2d(dst, &x_map, &x_full[s], (2 * u + st) * kTcBK, mt * kTcBT);
+                    else tma_load_2d(dst, &t_map, &x_full[s], 0, mt * kTcBT);
+                    if (++s == SX) { s = 0; ph ^= 1; }
+                }
             }
         }
-    a_done:
-        for (int i = 0; i < SA; ++i) {
+    x_done:
+        for (int i = 0; i < SX; ++i) {
             int local = 0;
-            if (armed[i] >= 0) (void)mbar_wait(&a_full[i], (uint32_t)armed[i], &local);
-        }
-    } else if (warp == 2 && lane == 0) {
-        // ---------------------------------------------------------- packed-weight producer
-        tma_prefetch_desc(&p_map);
-        int armed[SP];
-        for (int i = 0; i < SP; ++i) armed[i] = -1;
-        uint32_t s = 0, ph = 0;
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-            const int nt = tile / p.tiles_m;
-            for (int g = 0; g < G; ++g) {
-                if (!mbar_wait(&p_empty[s], ph ^ 1, abort)) goto p_done;
-                mbar_arrive_expect_tx(&p_full[s], L::kPBytes);
-                armed[s] = (int)ph;
-                tma_load_2d(smem + L::kOffP + s * L::kPBytes, &p_map, &p_full[s], g * 16 * BITS, nt * kTcBN);
-                if (++s == SP) { s = 0; ph ^= 1; }
-            }
-        }
-    p_done:
-        for (int i = 0; i < SP; ++i) {
-            int local = 0;
-            if (armed[i] >= 0) (void)mbar_wait(&p_full[i], (uint32_t)armed[i], &local);
+            if (armed[i] >= 0) (void)mbar_wait(&x_full[i], (uint32_t)armed[i], &local);
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc = umma_idesc_bf16(128, kTcBN);
-        uint32_t sa = 0, pa = 0, sb = 0, pb = 0, acc_ph = 0;
+        constexpr uint32_t idesc = umma_idesc_bf16(kTcBW, kTcBT);
+        uint32_t sa = 0, pa = 0, sx = 0, px = 0, unit = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-            if (!mbar_wait(acc_empty, acc_ph ^ 1, abort)) goto m_done;
-            acc_ph ^= 1;
-            tc_fence_after();
-            for (int kb = 0; kb < KB; ++kb) {
-                if (!mbar_wait(&a_full[sa], pa, abort)) goto m_done;
-                if (!mbar_wait(&b_full[sb], pb, abort)) goto m_done;
+            for (int u = 0; u < U; ++u, ++unit) {
+                const uint32_t tb = unit & 1, tph = (unit >> 1) & 1;
+                if (!mbar_wait(&t_empty[tb], tph ^ 1, abort)) goto m_done;
                 tc_fence_after();
-                const uint32_t a_base = smem_u32(smem + L::kOffA + sa * L::kABytes);
-                const uint32_t b_base = smem_u32(smem + L::kOffB + sb * L::kBBytes);
-                const int nk = (kb < KBm) ? kTcBK / 16 : p.rank / 16;
-                for (int k = 0; k < nk; ++k) {
-                    const uint64_t bd = umma_desc_sw128(b_base + k * 32, 1024);
-                    const uint64_t ad0 = umma_desc_sw128(a_base + k * 32, 1024);
-                    const uint64_t ad1 = umma_desc_sw128(a_base + 128 * 128 + k * 32, 1024);
-                    const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-                    umma_bf16(tmem, ad0, bd, idesc, acc);
-                    umma_bf16(tmem + kTcBN, ad1, bd, idesc, acc);
+                const uint32_t d = tmem + kTmemT0 + tb * kTcBT;
+                const int nst = (u < G) ? 2 : 1;
+                const int nk = (u < G) ? kTcBK / 16 : p.rank / 16;
+                for (int st = 0; st < nst; ++st) {
+                    if (!mbar_wait(&a_full[sa], pa, abort)) goto m_done;
+                    if (!mbar_wait(&x_full[sx], px, abort)) goto m_done;
+                    tc_fence_after();
+                    const uint32_t a = tmem + kTmemA + sa * (kTcBK / 2);
+                    const uint32_t b_base = smem_u32(smem + L::kOffX + sx * L::kXBytes);
+                    for (int k = 0; k < nk; ++k) {
+                        const uint64_t bd = umma_desc_sw128(b_base + k * 32, 1024);
+                        umma_bf16_ts(d, a + k * 8, bd, idesc, (st > 0 || k > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&a_empty[sa]);
+                    umma_commit(&x_empty[sx]);
+                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                    if (++sx == SX) { sx = 0; px ^= 1; }
                 }
-                umma_commit(&a_empty[sa]);
-                umma_commit(&b_empty[sb]);
-                if (++sa == SA) { sa = 0; pa ^= 1; }
-                if (++sb == SB) { sb = 0; pb ^= 1; }
+                umma_commit(&t_full[tb]);
             }
-            umma_commit(acc_full);
         }
     m_done:
         {
@@ -263,145 +299,136 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
             int local = 0;
             (void)mbar_wait(drain, 0, &local);
         }
-    } else if (warp >= kTcFirstDequantWarp) {
-        // ---------------------------------------------------------- dequant + epilogue
-        const int e = warp - kTcFirstDequantWarp;
-        const int nl = e * 32 + lane;                    // weight row inside the tile
-        const int quarter = warp & 3;                    // TMEM lanes this warp may access
-        const int half = e >> 2;                         // token half = accumulator
-        uint32_t sp = 0, pp = 0, sb = 0, pb = 0, acc_ph = 0;
+    } else if (warp >= kTcUnpackWarp0 && warp < kTcPromoteWarp0) {
+        // ---------------------------------------------------------- unpack codes into TMEM
+        const int quarter = warp & 3;
+        const int row_local = quarter * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        const int64_t row_bytes = p.K * BITS / 8;
+        uint32_t sa = 0, pa = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-            const int mt = tile % p.tiles_m, nt = tile / p.tiles_m;
-            const int64_t n = (int64_t)nt * kTcBN + nl;
+            const int nt = tile / p.tiles_m;
+            const int64_t n = (int64_t)nt * kTcBW + row_local;
             const bool row_ok = n < p.N;
-            const float *srow = p.scales + (row_ok ? n : 0) * (int64_t)G;
-            float step_next = row_ok ? __ldg(srow) : 0.0f;
+            const uint8_t *src = p.packed + (row_ok ? n : 0) * row_bytes;
+            uint32_t w0[NWG], w1[NWG], w2[NWG];
+            load_group<BITS>(src, row_ok && G > 0, w1);
+            load_group<BITS>(src + 16 * BITS, row_ok && G > 1, w2);
             for (int g = 0; g < G; ++g) {
-                const float step = step_next;
-                if (g + 1 < G) step_next = row_ok ? __ldg(srow + g + 1) : 0.0f;
-                if (!warp_wait(&p_full[sp], pp, abort)) goto d_done;
-                uint32_t w[4 * BITS + 1];
-                {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(smem + L::kOffP + sp * L::kPBytes + nl * 16 * BITS);
 #pragma unroll
-                    for (int i = 0; i < BITS; ++i) {
-                        const uint4 v = src[i];
-                        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-                    }
-                    w[4 * BITS] = 0;
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&p_empty[sp]);
-                if (++sp == SP) { sp = 0; pp ^= 1; }
-                // dequant = (c - 2^(b-1)) * step = f * S - T with f = 1 + c/128, S = 128 step
-                const float S = __fmul_rn(step, 128.0f);
-                const float T = __fmul_rn(S, 1.0f + (float)kHalf / 128.0f);
-                const int sw = nl & 7;
+                for (int i = 0; i < NWG; ++i) { w0[i] = w1[i]; w1[i] = w2[i]; }
+                load_group<BITS>(src + (int64_t)(g + 2) * 16 * BITS, row_ok && g + 2 < G, w2);
                 bool ok = true;
                 static_for<2>([&](auto hh) {
                     constexpr int h = decltype(hh)::value;
                     if (!ok) return;
-                    if (!warp_wait(&b_empty[sb], pb ^ 1, abort)) { ok = false; return; }
-                    uint8_t *row = smem + L::kOffB + sb * L::kBBytes + (nl >> 3) * 1024 + (nl & 7) * 128;
-                    static_for<8>([&](auto cc) {
-                        constexpr int c = decltype(cc)::value;
-                        uint32_t lo, hi;
-                        tc_block_be<BITS, 8 * h + c>(w, lo, hi);
-                        float f[8];
-                        static_for<8>([&](auto ii) {
-                            constexpr int i = decltype(ii)::value;
-                            f[i] = fmaf(tc_code_f32<BITS, i>(lo, hi), S, -T);
-                        });
-                        uint4 o;
-                        o.x = pack_bf16x2(f[0], f[1]);
-                        o.y = pack_bf16x2(f[2], f[3]);
-                        o.z = pack_bf16x2(f[4], f[5]);
-                        o.w = pack_bf16x2(f[6], f[7]);
-                        *reinterpret_cast<uint4 *>(row + ((c ^ sw) << 4)) = o;
-                    });
-                    fence_proxy_async_smem();
+                    uint32_t q[32];
+                    unpack_half<BITS, h>(w0, q);
+                    if (!warp_wait(&a_empty[sa], pa ^ 1, abort)) { ok = false; return; }
+                    tmem_st_32x32b_x32(tmem + lane_addr + kTmemA + sa * (kTcBK / 2), q);
+                    tmem_wait_st();
+                    tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&b_full[sb]);
-                    if (++sb == SB) { sb = 0; pb ^= 1; }
+                    if (lane == 0) mbar_arrive(&a_full[sa]);
+                    if (++sa == SA) { sa = 0; pa ^= 1; }
                 });
-                if (!ok) goto d_done;
+                if (!ok) goto u_done;
             }
             if (p.rank > 0) {
-                // low-rank stage: B[n][j] = L2[j][n] for j < rank, zero up to 64
-                if (!warp_wait(&b_empty[sb], pb ^ 1, abort)) goto d_done;
-                uint8_t *row = smem + L::kOffB + sb * L::kBBytes + (nl >> 3) * 1024 + (nl & 7) * 128;
-                const int sw = nl & 7;
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t v[4] = {0u, 0u, 0u, 0u};
-                    if (row_ok && 8 * c < p.rank) {
+                // low-rank unit: A[n][j] = L2[j][n] for j < rank, zero up to 64
+                uint32_t q[32];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const uint32_t a = __ldg(p.L2 + (int64_t)(8 * c + 2 * i) * p.N + n);
-                            const uint32_t b = __ldg(p.L2 + (int64_t)(8 * c + 2 * i + 1) * p.N + n);
-                            v[i] = a | (b << 16);
+                for (int i = 0; i < 32; ++i) {
+                    uint32_t v = 0;
+                    if (row_ok && 2 * i < p.rank) {
+                        const uint32_t a = __ldg(p.L2 + (int64_t)(2 * i) * p.N + n);
+                        const uint32_t b = __ldg(p.L2 + (int64_t)(2 * i + 1) * p.N + n);
+                        v = a | (b << 16);
+                    }
+                    q[i] = v;
+                }
+                if (!warp_wait(&a_empty[sa], pa ^ 1, abort)) goto u_done;
+                tmem_st_32x32b_x32(tmem + lane_addr + kTmemA + sa * (kTcBK / 2), q);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a_full[sa]);
+                if (++sa == SA) { sa = 0; pa ^= 1; }
+            }
+        }
+    u_done:;
+    } else if (warp >= kTcPromoteWarp0) {
+        // ---------------------------------------------------------- promotion + epilogue
+        const int quarter = warp & 3;
+        const int row_local = quarter * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        uint32_t unit = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+            const int mt = tile % p.tiles_m, nt = tile / p.tiles_m;
+            const int64_t n = (int64_t)nt * kTcBW + row_local;
+            const bool row_ok = n < p.N;
+            const float *srow = p.scales + (row_ok ? n : 0) * (int64_t)G;
+            float s_next0 = (row_ok && G > 0) ? __ldg(srow) : 0.0f;
+            float s_next1 = (row_ok && G > 1) ? __ldg(srow + 1) : 0.0f;
+            for (int u = 0; u < U; ++u, ++unit) {
+                float s;
+                if (u < G) {
+                    s = s_next0;
+                    s_next0 = s_next1;
+                    s_next1 = (row_ok && u + 2 < G) ? __ldg(srow + u + 2) : 0.0f;
+                } else {
+                    s = 1.0f;
+                }
+                const uint32_t tb = unit & 1, tph = (unit >> 1) & 1;
+                if (!warp_wait(&t_full[tb], tph, abort)) goto p_done;
+                tc_fence_after();
+                const uint32_t t_addr = tmem + lane_addr + kTmemT0 + tb * kTcBT;
+                const uint32_t r_addr = tmem + lane_addr + kTmemR;
+                for (int c = 0; c < kTcBT / 32; ++c) {
+                    uint32_t tv[32], rv[32];
+                    tmem_ld_32x32b_x32(t_addr + c * 32, tv);
+                    if (u > 0) tmem_ld_32x32b_x32(r_addr + c * 32, rv);
+                    tmem_wait_ld();
+                    if (u == 0) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) rv[i] = __float_as_uint(__uint_as_float(tv[i]) * s);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            float d0, d1;
+                            ffma2(d0, d1, __uint_as_float(tv[i]), __uint_as_float(tv[i + 1]), s, s,
+                                  __uint_as_float(rv[i]), __uint_as_float(rv[i + 1]));
+                            rv[i] = __float_as_uint(d0);
+                            rv[i + 1] = __float_as_uint(d1);
                         }
                     }
-                    *reinterpret_cast<uint4 *>(row + ((c ^ sw) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+                    tmem_st_32x32b_x32(r_addr + c * 32, rv);
                 }
-                fence_proxy_async_smem();
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&b_full[sb]);
-                if (++sb == SB) { sb = 0; pb ^= 1; }
+                if (lane == 0) mbar_arrive(&t_empty[tb]);
             }
             // ------------------------------------------------------ epilogue
-            if (!warp_wait(acc_full, acc_ph, abort)) goto d_done;
-            acc_ph ^= 1;
-            tc_fence_after();
             {
-                const int64_t m = (int64_t)mt * kTcBM + half * 128 + quarter * 32 + lane;
-                const bool vec = (p.N % 8) == 0;
-                for (int cc = 0; cc < kTcBN / 32; ++cc) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + half * kTcBN + cc * 32, r);
+                const float bn = (row_ok && p.bias) ? bf16_bits_to_f32(__ldg(p.bias + n)) : 0.0f;
+                const uint32_t r_addr = tmem + lane_addr + kTmemR;
+                for (int c = 0; c < kTcBT / 32; ++c) {
+                    uint32_t rv[32];
+                    tmem_ld_32x32b_x32(r_addr + c * 32, rv);
                     tmem_wait_ld();
-                    const int64_t nb = (int64_t)nt * kTcBN + cc * 32;
-                    if (m < p.M) {
-                        uint16_t *yrow = p.y + m * p.N;
+                    const int64_t m0 = (int64_t)mt * kTcBT + c * 32;
+                    if (row_ok) {
 #pragma unroll
-                        for (int j = 0; j < 32; j += 8) {
-                            float v[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[j + i]);
-                            const int64_t n0 = nb + j;
-                            if (vec && n0 + 8 <= p.N) {
-                                if (p.bias) {
-                                    const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(p.bias + n0));
-                                    const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-                                    for (int i = 0; i < 4; ++i) {
-                                        v[2 * i] += bf16_bits_to_f32(bw[i] & 0xFFFFu);
-                                        v[2 * i + 1] += bf16_bits_to_f32(bw[i] >> 16);
-                                    }
-                                }
-                                uint4 o;
-                                o.x = pack_bf16x2(v[0], v[1]);
-                                o.y = pack_bf16x2(v[2], v[3]);
-                                o.z = pack_bf16x2(v[4], v[5]);
-                                o.w = pack_bf16x2(v[6], v[7]);
-                                *reinterpret_cast<uint4 *>(yrow + n0) = o;
-                            } else {
-                                for (int i = 0; i < 8; ++i) {
-                                    if (n0 + i < p.N) {
-                                        float a = v[i];
-                                        if (p.bias) a += bf16_bits_to_f32(__ldg(p.bias + n0 + i));
-                                        yrow[n0 + i] = __bfloat16_as_ushort(__float2bfloat16_rn(a));
-                                    }
-                                }
-                            }
+                        for (int j = 0; j < 32; ++j) {
+                            if (m0 + j < p.M)
+                                p.y[(m0 + j) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(rv[j]) + bn));
                         }
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
         }
-    d_done:;
+    p_done:;
     }
 
     tc_fence_before();
