@@ -90,7 +90,7 @@ class ClockSampler:
         0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.005):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
         self._period = period_s
@@ -199,15 +199,14 @@ def oracle_sample(lins_host, rows_per_linear: int, pack_rows: int):
 
 def cpu_baseline(lins_host, budget_s: float = 12.0):
     import oracle
-    f, p, t = oracle_sample(lins_host, 4, 1024)          # calibration
-    scale = max(1.0, budget_s / max(t, 1e-3))
-    rows = max(4, min(512, int(4 * scale)))
-    prow = max(256, min(3072, int(1024 * scale)))
+    prow = min(lin["N"] for lin in lins_host)
+    f, p, t = oracle_sample(lins_host, 8, prow)          # calibration
+    rows = int(max(8, min(2048, 8 * budget_s / max(t, 1e-3))))
     f, p, t = oracle_sample(lins_host, rows, prow)
     return {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
             "sample": (f"C oracle (fp32 quantize+pack, fp64 linear with the rank-32 branch) on {prow} weight rows "
-                       f"of each of the 3 residuals x {rows} token rows: {f / 1e9:.2f} GFLOP in {t:.1f} s; "
-                       f"oracle pack rate {p / t / 1e9:.4f} Gparam/s (pack+dequant+linear wall time)")}
+                       f"of each of the 3 residuals x {rows} token rows: {f / 1e9:.2f} GFLOP in {t:.1f} s "
+                       f"(pack+dequant+linear wall time)")}
 
 
 def reference_arm(args):

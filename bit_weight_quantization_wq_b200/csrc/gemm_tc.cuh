@@ -15,19 +15,21 @@
 // Orientation: D = W_q x^T, so TMEM lanes are weight rows and columns are tokens; the
 // per-group step is then one scalar per lane.
 // One persistent CTA per SM walks 128 x 128 tiles (128 weight rows x 128 tokens).
-// TMEM (512 columns): T0, T1 = per-group partials (double-buffered, 128 columns each),
-// R = running sum (128), A = 4 stages of codes (32 columns = 64 k each).
-// Warp roles (384 threads):
+// TMEM (512 columns): T0, T1 = per-group partials (double-buffered, 128 columns each) and
+// 8 stages of codes (32 columns = 64 k each).
+// Warp roles (512 threads):
 //   warp 0      TMA producer of x tiles (128 tokens x 64 k bf16, 128B swizzle, 16 KB/stage)
 //   warp 1      TMEM allocator; one thread issues tcgen05.mma (A = codes from TMEM,
 //               B = x from shared memory, M=128 N=128 K=16) into T
-//   warps 4-7   unpack: one weight row per thread; packed bytes come from global memory
-//               straight into registers (two groups ahead), become bf16 pairs of exact q
-//               and are written to the A stage with tcgen05.st
-//   warps 8-11  promotion: R += step * T per group (fp32, two lanes per instruction), then the
-//               epilogue (+ bias, round once to bf16, store y)
-// Low-rank branch: one more unit per tile with A = L2^T (bf16 from global) and B = the
-// t = bf16(x L1) tile, promoted with scale 1 into the same R.
+//   warp 2      TMA producer of packed-weight tiles (128 rows x one group, 16*b bytes a row)
+//   warps 4-7   unpack: one weight row per thread; bf16 pairs of exact q written to the A
+//               stage with tcgen05.st
+//   warps 8-15  promotion: R += step * T per group (fp32, two lanes per instruction) with R in
+//               registers (two warps per TMEM lane quarter, 64 columns each), then the epilogue
+//               (+ bias, round once to bf16, store y)
+// Low-rank branch: one more unit per tile with B = [t_hi | t_lo] (t = x L1 split into two
+// bf16 terms by lowrank_prepass_kernel) and A = [L2^T | L2^T] (bf16 from global), promoted
+// with scale 1 into the same R; the split keeps t's rounding out of the result.
 //
 // Every wait is bounded (see common.cuh). On a timeout the roles stop, the producer waits
 // (bounded) for its copies in flight, the MMA thread for its MMAs, and TMEM is freed.
@@ -44,26 +46,32 @@ constexpr int kTcBW = 128;                // weight rows per tile (MMA M)
 constexpr int kTcBT = 128;                // tokens per tile (MMA N)
 constexpr int kTcBK = 64;                 // k per x stage / A stage
 constexpr int kTcStagesX = 6;
-constexpr int kTcStagesA = 4;
-constexpr int kTcThreads = 384;
+constexpr int kTcStagesA = 8;
+constexpr int kTcThreads = 512;
 constexpr int kTcUnpackWarp0 = 4;
 constexpr int kTcPromoteWarp0 = 8;
+constexpr int kTcPromoteWarps = 8;
 constexpr uint32_t kTcTmemCols = 512;
-constexpr uint32_t kTmemT0 = 0, kTmemR = 256, kTmemA = 384;
-constexpr int kTStride = 64;              // row stride (elements) of the low-rank t buffer
+constexpr uint32_t kTmemT0 = 0, kTmemA = 256;
+constexpr int kTStride = 128;             // row stride (elements) of the low-rank [t_hi | t_lo] buffer
 
+template <int BITS> struct TcStagesP { static constexpr int value = BITS <= 4 ? 8 : 6; };
+
+template <int BITS>
 struct TcLayout {
+    static constexpr int kSP = TcStagesP<BITS>::value;
     static constexpr uint32_t kXBytes = kTcBT * kTcBK * 2;          // 16 KB
+    static constexpr uint32_t kPBytes = kTcBW * 16 * BITS;          // 128 rows x one group
     static constexpr uint32_t kOffX = 0;
-    static constexpr uint32_t kOffBar = kOffX + kTcStagesX * kXBytes;
-    static constexpr uint32_t kNumBars = 2 * kTcStagesX + 2 * kTcStagesA + 4 + 1;
+    static constexpr uint32_t kOffP = kOffX + kTcStagesX * kXBytes;
+    static constexpr uint32_t kOffBar = kOffP + kSP * kPBytes;
+    static constexpr uint32_t kNumBars = 2 * kTcStagesX + 2 * kSP + 2 * kTcStagesA + 4 + 1;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kBytes = kOffMisc + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;               // slack to align the base to 1024 B
 };
 
 struct TcParams {
-    const uint8_t *packed;    // N x K*bits/8
     const float *scales;      // N x K/128
     const uint16_t *L2;       // rank x N bf16 or null
     const uint16_t *bias;     // N bf16 or null
@@ -72,6 +80,9 @@ struct TcParams {
     int rank;
     int tiles_m, tiles_n;
 };
+
+// k stages (64 wide) of the low-rank unit: [t_hi | t_lo] has 2 * rank columns.
+__host__ __device__ constexpr int lowrank_stages(int rank) { return (2 * rank + kTcBK - 1) / kTcBK; }
 
 template <int I> struct Int { static constexpr int value = I; };
 template <int N, int I = 0, class F>
@@ -187,28 +198,19 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 template <int BITS>
-__device__ __forceinline__ void load_group(const uint8_t *src, bool ok, uint32_t (&w)[4 * BITS + 1]) {
-#pragma unroll
-    for (int i = 0; i < BITS; ++i) {
-        const uint4 v = ok ? __ldg(reinterpret_cast<const uint4 *>(src) + i) : make_uint4(0, 0, 0, 0);
-        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-    }
-    w[4 * BITS] = 0;
-}
-
-template <int BITS>
 __global__ void __launch_bounds__(kTcThreads, 1)
-tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap t_map,
-                 const TcParams p) {
-    using L = TcLayout;
-    constexpr int SX = kTcStagesX, SA = kTcStagesA;
+tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap p_map,
+                 const __grid_constant__ CUtensorMap t_map, const TcParams p) {
+    using L = TcLayout<BITS>;
+    constexpr int SX = kTcStagesX, SA = kTcStagesA, SP = L::kSP;
     constexpr int NWG = 4 * BITS + 1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
     uint64_t *x_full = bars, *x_empty = x_full + SX;
-    uint64_t *a_full = x_empty + SX, *a_empty = a_full + SA;
+    uint64_t *p_full = x_empty + SX, *p_empty = p_full + SP;
+    uint64_t *a_full = p_empty + SP, *a_empty = a_full + SA;
     uint64_t *t_full = a_empty + SA, *t_empty = t_full + 2, *drain = t_empty + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
@@ -216,8 +218,9 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < SX; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
+        for (int i = 0; i < SP; ++i) { mbar_init(&p_full[i], 1); mbar_init(&p_empty[i], 4); }
         for (int i = 0; i < SA; ++i) { mbar_init(&a_full[i], 4); mbar_init(&a_empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&t_full[i], 1); mbar_init(&t_empty[i], 4); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&t_full[i], 1); mbar_init(&t_empty[i], kTcPromoteWarps); }
         mbar_init(drain, 1);
         *abort = 0;
         fence_barrier_init();
@@ -245,14 +248,14 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int mt = tile % p.tiles_m;
             for (int u = 0; u < U; ++u) {
-                const int nst = (u < G) ? 2 : 1;
+                const int nst = (u < G) ? 2 : lowrank_stages(p.rank);
                 for (int st = 0; st < nst; ++st) {
                     if (!mbar_wait(&x_empty[s], ph ^ 1, abort)) goto x_done;
                     mbar_arrive_expect_tx(&x_full[s], L::kXBytes);
                     armed[s] = (int)ph;
                     uint8_t *dst = smem + L::kOffX + s * L::kXBytes;
                     if (u < G) tma_load_2d(dst, &x_map, &x_full[s], (2 * u + st) * kTcBK, mt * kTcBT);
-                    else tma_load_2d(dst, &t_map, &x_full[s], 0, mt * kTcBT);
+                    else tma_load_2d(dst, &t_map, &x_full[s], st * kTcBK, mt * kTcBT);
                     if (++s == SX) { s = 0; ph ^= 1; }
                 }
             }
@@ -261,6 +264,27 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         for (int i = 0; i < SX; ++i) {
             int local = 0;
             if (armed[i] >= 0) (void)mbar_wait(&x_full[i], (uint32_t)armed[i], &local);
+        }
+    } else if (warp == 2 && lane == 0) {
+        // ---------------------------------------------------------- packed-weight producer
+        tma_prefetch_desc(&p_map);
+        int armed[SP];
+        for (int i = 0; i < SP; ++i) armed[i] = -1;
+        uint32_t s = 0, ph = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+            const int nt = tile / p.tiles_m;
+            for (int g = 0; g < G; ++g) {
+                if (!mbar_wait(&p_empty[s], ph ^ 1, abort)) goto p_done;
+                mbar_arrive_expect_tx(&p_full[s], L::kPBytes);
+                armed[s] = (int)ph;
+                tma_load_2d(smem + L::kOffP + s * L::kPBytes, &p_map, &p_full[s], g * 16 * BITS, nt * kTcBW);
+                if (++s == SP) { s = 0; ph ^= 1; }
+            }
+        }
+    p_done:
+        for (int i = 0; i < SP; ++i) {
+            int local = 0;
+            if (armed[i] >= 0) (void)mbar_wait(&p_full[i], (uint32_t)armed[i], &local);
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------------------------------------------------- MMA issuer
@@ -272,9 +296,9 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                 if (!mbar_wait(&t_empty[tb], tph ^ 1, abort)) goto m_done;
                 tc_fence_after();
                 const uint32_t d = tmem + kTmemT0 + tb * kTcBT;
-                const int nst = (u < G) ? 2 : 1;
-                const int nk = (u < G) ? kTcBK / 16 : p.rank / 16;
+                const int nst = (u < G) ? 2 : lowrank_stages(p.rank);
                 for (int st = 0; st < nst; ++st) {
+                    const int nk = (u < G) ? kTcBK / 16 : min(kTcBK, 2 * p.rank - st * kTcBK) / 16;
                     if (!mbar_wait(&a_full[sa], pa, abort)) goto m_done;
                     if (!mbar_wait(&x_full[sx], px, abort)) goto m_done;
                     tc_fence_after();
@@ -304,27 +328,34 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         const int quarter = warp & 3;
         const int row_local = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        const int64_t row_bytes = p.K * BITS / 8;
-        uint32_t sa = 0, pa = 0;
+        uint32_t sa = 0, pa = 0, sp = 0, pp = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int nt = tile / p.tiles_m;
             const int64_t n = (int64_t)nt * kTcBW + row_local;
             const bool row_ok = n < p.N;
-            const uint8_t *src = p.packed + (row_ok ? n : 0) * row_bytes;
-            uint32_t w0[NWG], w1[NWG], w2[NWG];
-            load_group<BITS>(src, row_ok && G > 0, w1);
-            load_group<BITS>(src + 16 * BITS, row_ok && G > 1, w2);
             for (int g = 0; g < G; ++g) {
+                if (!warp_wait(&p_full[sp], pp, abort)) goto u_done;
+                uint32_t w[NWG];
+                {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(smem + L::kOffP + sp * L::kPBytes +
+                                                                        row_local * 16 * BITS);
 #pragma unroll
-                for (int i = 0; i < NWG; ++i) { w0[i] = w1[i]; w1[i] = w2[i]; }
-                load_group<BITS>(src + (int64_t)(g + 2) * 16 * BITS, row_ok && g + 2 < G, w2);
+                    for (int i = 0; i < BITS; ++i) {
+                        const uint4 v = src[i];
+                        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+                    }
+                    w[4 * BITS] = 0;
+                }
+                const uint32_t sp_used = sp;
+                if (++sp == SP) { sp = 0; pp ^= 1; }
                 bool ok = true;
                 static_for<2>([&](auto hh) {
                     constexpr int h = decltype(hh)::value;
                     if (!ok) return;
                     uint32_t q[32];
-                    unpack_half<BITS, h>(w0, q);
+                    unpack_half<BITS, h>(w, q);
                     if (!warp_wait(&a_empty[sa], pa ^ 1, abort)) { ok = false; return; }
+                    tc_fence_after();        // order the store after the MMAs that read this stage
                     tmem_st_32x32b_x32(tmem + lane_addr + kTmemA + sa * (kTcBK / 2), q);
                     tmem_wait_st();
                     tc_fence_before();
@@ -332,103 +363,105 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                     if (lane == 0) mbar_arrive(&a_full[sa]);
                     if (++sa == SA) { sa = 0; pa ^= 1; }
                 });
+                // the stage's bytes have been consumed by every lane (both halves are in TMEM):
+                // only now may the producer overwrite it
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_empty[sp_used]);
                 if (!ok) goto u_done;
             }
             if (p.rank > 0) {
-                // low-rank unit: A[n][j] = L2[j][n] for j < rank, zero up to 64
-                uint32_t q[32];
+                // low-rank unit: A[n][k] = L2[k mod rank][n] for k < 2 rank (both halves of
+                // [t_hi | t_lo] meet the same L2), zero beyond
+                const int nst = lowrank_stages(p.rank);
+                for (int st = 0; st < nst; ++st) {
+                    uint32_t q[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    uint32_t v = 0;
-                    if (row_ok && 2 * i < p.rank) {
-                        const uint32_t a = __ldg(p.L2 + (int64_t)(2 * i) * p.N + n);
-                        const uint32_t b = __ldg(p.L2 + (int64_t)(2 * i + 1) * p.N + n);
-                        v = a | (b << 16);
+                    for (int i = 0; i < 32; ++i) {
+                        const int k = st * kTcBK + 2 * i;
+                        uint32_t v = 0;
+                        if (row_ok && k < 2 * p.rank) {
+                            const int j = k % p.rank;
+                            const uint32_t a = __ldg(p.L2 + (int64_t)j * p.N + n);
+                            const uint32_t b = __ldg(p.L2 + (int64_t)(j + 1) * p.N + n);
+                            v = a | (b << 16);
+                        }
+                        q[i] = v;
                     }
-                    q[i] = v;
+                    if (!warp_wait(&a_empty[sa], pa ^ 1, abort)) goto u_done;
+                    tc_fence_after();
+                    tmem_st_32x32b_x32(tmem + lane_addr + kTmemA + sa * (kTcBK / 2), q);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&a_full[sa]);
+                    if (++sa == SA) { sa = 0; pa ^= 1; }
                 }
-                if (!warp_wait(&a_empty[sa], pa ^ 1, abort)) goto u_done;
-                tmem_st_32x32b_x32(tmem + lane_addr + kTmemA + sa * (kTcBK / 2), q);
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[sa]);
-                if (++sa == SA) { sa = 0; pa ^= 1; }
             }
         }
     u_done:;
     } else if (warp >= kTcPromoteWarp0) {
         // ---------------------------------------------------------- promotion + epilogue
         const int quarter = warp & 3;
+        const int colh = (warp - kTcPromoteWarp0) >> 2;            // which 64 token columns
         const int row_local = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        constexpr int kPre = 4;                                     // scale prefetch distance
         uint32_t unit = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int mt = tile % p.tiles_m, nt = tile / p.tiles_m;
             const int64_t n = (int64_t)nt * kTcBW + row_local;
             const bool row_ok = n < p.N;
             const float *srow = p.scales + (row_ok ? n : 0) * (int64_t)G;
-            float s_next0 = (row_ok && G > 0) ? __ldg(srow) : 0.0f;
-            float s_next1 = (row_ok && G > 1) ? __ldg(srow + 1) : 0.0f;
+            float sq[kPre];
+#pragma unroll
+            for (int i = 0; i < kPre; ++i) sq[i] = (row_ok && i < G) ? __ldg(srow + i) : 0.0f;
+            float R[64];
             for (int u = 0; u < U; ++u, ++unit) {
-                float s;
+                float s = 1.0f;
                 if (u < G) {
-                    s = s_next0;
-                    s_next0 = s_next1;
-                    s_next1 = (row_ok && u + 2 < G) ? __ldg(srow + u + 2) : 0.0f;
-                } else {
-                    s = 1.0f;
+                    s = sq[0];
+#pragma unroll
+                    for (int i = 0; i + 1 < kPre; ++i) sq[i] = sq[i + 1];
+                    sq[kPre - 1] = (row_ok && u + kPre < G) ? __ldg(srow + u + kPre) : 0.0f;
                 }
                 const uint32_t tb = unit & 1, tph = (unit >> 1) & 1;
-                if (!warp_wait(&t_full[tb], tph, abort)) goto p_done;
+                if (!warp_wait(&t_full[tb], tph, abort)) goto pr_done;
                 tc_fence_after();
-                const uint32_t t_addr = tmem + lane_addr + kTmemT0 + tb * kTcBT;
-                const uint32_t r_addr = tmem + lane_addr + kTmemR;
-                for (int c = 0; c < kTcBT / 32; ++c) {
-                    uint32_t tv[32], rv[32];
-                    tmem_ld_32x32b_x32(t_addr + c * 32, tv);
-                    if (u > 0) tmem_ld_32x32b_x32(r_addr + c * 32, rv);
+                const uint32_t t_addr = tmem + lane_addr + kTmemT0 + tb * kTcBT + colh * 64;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t tv[32];
+                    tmem_ld_32x32b_x32(t_addr + 32 * hf, tv);
                     tmem_wait_ld();
+                    if (hf == 1) {
+                        // both halves of T are in registers: hand the buffer back to the MMA
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&t_empty[tb]);
+                    }
                     if (u == 0) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) rv[i] = __float_as_uint(__uint_as_float(tv[i]) * s);
+                        for (int i = 0; i < 32; ++i) R[32 * hf + i] = __uint_as_float(tv[i]) * s;
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
-                            float d0, d1;
-                            ffma2(d0, d1, __uint_as_float(tv[i]), __uint_as_float(tv[i + 1]), s, s,
-                                  __uint_as_float(rv[i]), __uint_as_float(rv[i + 1]));
-                            rv[i] = __float_as_uint(d0);
-                            rv[i + 1] = __float_as_uint(d1);
-                        }
+                        for (int i = 0; i < 32; i += 2)
+                            ffma2(R[32 * hf + i], R[32 * hf + i + 1], __uint_as_float(tv[i]), __uint_as_float(tv[i + 1]),
+                                  s, s, R[32 * hf + i], R[32 * hf + i + 1]);
                     }
-                    tmem_st_32x32b_x32(r_addr + c * 32, rv);
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&t_empty[tb]);
             }
             // ------------------------------------------------------ epilogue
-            {
-                const float bn = (row_ok && p.bias) ? bf16_bits_to_f32(__ldg(p.bias + n)) : 0.0f;
-                const uint32_t r_addr = tmem + lane_addr + kTmemR;
-                for (int c = 0; c < kTcBT / 32; ++c) {
-                    uint32_t rv[32];
-                    tmem_ld_32x32b_x32(r_addr + c * 32, rv);
-                    tmem_wait_ld();
-                    const int64_t m0 = (int64_t)mt * kTcBT + c * 32;
-                    if (row_ok) {
+            if (row_ok) {
+                const float bn = p.bias ? bf16_bits_to_f32(__ldg(p.bias + n)) : 0.0f;
+                const int64_t m0 = (int64_t)mt * kTcBT + colh * 64;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            if (m0 + j < p.M)
-                                p.y[(m0 + j) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(rv[j]) + bn));
-                        }
-                    }
+                for (int j = 0; j < 64; ++j) {
+                    if (m0 + j < p.M)
+                        p.y[(m0 + j) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(R[j] + bn));
                 }
             }
         }
-    p_done:;
+    pr_done:;
     }
 
     tc_fence_before();
@@ -441,8 +474,9 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
 }
 
 // ---------------------------------------------------------------------------------------
-// t = bf16(x L1): M x R (R = rank, 16..64), stored with a row stride of kTStride = 64
-// elements (columns R..63 zero) so that one 64-wide TMA box covers a row exactly.
+// t = x L1 (M x R, R = rank 16..64) as two bf16 terms, t_hi = bf16(t) in columns [0, R) and
+// t_lo = bf16(t - t_hi) in [R, 2R), row stride kTStride = 128 (the rest zero), so that
+// 64-wide TMA boxes cover a row exactly.
 // x is read once; tensor cores via mma.m16n8k16.
 // grid (ceil(M/64), KS) with clusters of KS CTAs along K; a CTA owns 64 tokens (4 warps x
 // 16) and 1/KS of K; partial sums are added through distributed shared memory.
@@ -537,15 +571,21 @@ lowrank_prepass_kernel(const uint16_t *__restrict__ x, const uint16_t *__restric
         float v = 0.0f;
         for (uint32_t r = 0; r < KS; ++r) v += ld_cluster_f32(map_cluster_smem(base + 4u * e, r));
         const int64_t m = m0 + e / R;
-        if (m < M) t[m * kTStride + e % R] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        if (m < M) {
+            // two bf16 terms: t_hi = bf16(t) in column j, t_lo = bf16(t - t_hi) in column R + j
+            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+            t[m * kTStride + e % R] = __bfloat16_as_ushort(hi);
+            t[m * kTStride + R + e % R] = __bfloat16_as_ushort(lo);
+        }
     }
-    if constexpr (R < kTStride) {
-        // zero the padding columns so that the whole 64-wide row is defined
-        constexpr int kPad = kTStride - R;
+    if constexpr (2 * R < kTStride) {
+        // zero the padding columns so that the whole row is defined
+        constexpr int kPad = kTStride - 2 * R;
         if (split == 0) {
             for (int i = tid; i < 64 * kPad; i += 128) {
                 const int64_t m = m0 + i / kPad;
-                if (m < M) t[m * kTStride + R + i % kPad] = 0;
+                if (m < M) t[m * kTStride + 2 * R + i % kPad] = 0;
             }
         }
     }

@@ -197,8 +197,9 @@ wq_status make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base
 }
 
 template <int BITS>
-wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &tm, int sm_count, cudaStream_t st) {
-    using L = wq::TcLayout;
+wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &pm, const CUtensorMap &tm,
+                    int sm_count, cudaStream_t st) {
+    using L = wq::TcLayout<BITS>;
     static bool attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -209,7 +210,6 @@ wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &t
         attr_done[dev] = true;
     }
     wq::TcParams p{};
-    p.packed = a.packed;
     p.scales = a.scales;
     p.L2 = static_cast<const uint16_t *>(a.L2);
     p.bias = static_cast<const uint16_t *>(a.bias);
@@ -219,7 +219,7 @@ wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &t
     p.tiles_n = (int)((a.N + wq::kTcBW - 1) / wq::kTcBW);
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = std::min(tiles, sm_count);
-    wq::tc_linear_kernel<BITS><<<grid, wq::kTcThreads, L::kAlloc, st>>>(xm, tm, p);
+    wq::tc_linear_kernel<BITS><<<grid, wq::kTcThreads, L::kAlloc, st>>>(xm, pm, tm, p);
     return check_launch("tc_linear_kernel");
 }
 
@@ -252,9 +252,13 @@ wq_status tc_linear(const TcArgs &a, int sm_count, cudaStream_t st) {
     if (s != WQ_OK) return s;
     if (a.M > (int64_t)INT32_MAX || a.N > (int64_t)INT32_MAX || a.K > (int64_t)INT32_MAX)
         return fail(WQ_ERR_INVALID_ARG, "dimension above 2^31 on the tensor-core path");
-    CUtensorMap xm, tm;
+    CUtensorMap xm, pm, tm;
     if ((s = make_map_2d(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)a.K, (uint64_t)a.M,
                          (uint64_t)a.K * 2, wq::kTcBK, wq::kTcBT, CU_TENSOR_MAP_SWIZZLE_128B)) != WQ_OK)
+        return s;
+    const uint64_t row_bytes = (uint64_t)a.K * a.bits / 8;
+    if ((s = make_map_2d(&pm, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.packed, row_bytes, (uint64_t)a.N, row_bytes,
+                         16u * a.bits, wq::kTcBW, CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK)
         return s;
     tm = xm;
     if (a.rank > 0) {
@@ -271,11 +275,11 @@ wq_status tc_linear(const TcArgs &a, int sm_count, cudaStream_t st) {
             return s;
     }
     switch (a.bits) {
-        case 3: return launch_tc<3>(a, xm, tm, sm_count, st);
-        case 4: return launch_tc<4>(a, xm, tm, sm_count, st);
-        case 5: return launch_tc<5>(a, xm, tm, sm_count, st);
-        case 6: return launch_tc<6>(a, xm, tm, sm_count, st);
-        default: return launch_tc<7>(a, xm, tm, sm_count, st);
+        case 3: return launch_tc<3>(a, xm, pm, tm, sm_count, st);
+        case 4: return launch_tc<4>(a, xm, pm, tm, sm_count, st);
+        case 5: return launch_tc<5>(a, xm, pm, tm, sm_count, st);
+        case 6: return launch_tc<6>(a, xm, pm, tm, sm_count, st);
+        default: return launch_tc<7>(a, xm, pm, tm, sm_count, st);
     }
 }
 
