@@ -27,6 +27,11 @@
 //   warps 8-15  promotion: R += step * T per group (fp32, two lanes per instruction) with R in
 //               registers (two warps per TMEM lane quarter, 64 columns each), then the epilogue
 //               (+ bias, round once to bf16, store y)
+// Synchronization is per unit (one 128-k group, or the low-rank unit), not per k stage: the
+// single MMA-issuing thread pays ~140 cycles per mbarrier wait, so it waits once per unit on
+// ready[slot], which completes when the unit's x tiles have landed (TMA transaction bytes),
+// its codes are in TMEM (4 unpack warps) and its T buffer is free (8 promotion warps); one
+// commit per unit releases the slot (consumed[slot]) and another hands T to the promotion.
 // Low-rank branch: one more unit per tile with B = [t_hi | t_lo] (t = x L1 split into two
 // bf16 terms by lowrank_prepass_kernel) and A = [L2^T | L2^T] (bf16 from global), promoted
 // with scale 1 into the same R; the split keeps t's rounding out of the result.
@@ -45,8 +50,9 @@ namespace wq {
 constexpr int kTcBW = 128;                // weight rows per tile (MMA M)
 constexpr int kTcBT = 128;                // tokens per tile (MMA N)
 constexpr int kTcBK = 64;                 // k per x stage / A stage
-constexpr int kTcStagesX = 6;
-constexpr int kTcStagesA = 8;
+constexpr int kTcSlots = 4;               // units in flight (each: 2 x stages + 2 code stages)
+constexpr int kTcStagesX = 2 * kTcSlots;
+constexpr int kTcStagesA = 2 * kTcSlots;
 constexpr int kTcThreads = 512;
 constexpr int kTcUnpackWarp0 = 4;
 constexpr int kTcPromoteWarp0 = 8;
@@ -65,7 +71,7 @@ struct TcLayout {
     static constexpr uint32_t kOffX = 0;
     static constexpr uint32_t kOffP = kOffX + kTcStagesX * kXBytes;
     static constexpr uint32_t kOffBar = kOffP + kSP * kPBytes;
-    static constexpr uint32_t kNumBars = 2 * kTcStagesX + 2 * kSP + 2 * kTcStagesA + 4 + 1;
+    static constexpr uint32_t kNumBars = 2 * kTcSlots + 2 * kSP + 2 + 1;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kBytes = kOffMisc + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;               // slack to align the base to 1024 B
@@ -202,25 +208,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap p_map,
                  const __grid_constant__ CUtensorMap t_map, const TcParams p) {
     using L = TcLayout<BITS>;
-    constexpr int SX = kTcStagesX, SA = kTcStagesA, SP = L::kSP;
+    constexpr int SP = L::kSP;
     constexpr int NWG = 4 * BITS + 1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
-    uint64_t *x_full = bars, *x_empty = x_full + SX;
-    uint64_t *p_full = x_empty + SX, *p_empty = p_full + SP;
-    uint64_t *a_full = p_empty + SP, *a_empty = a_full + SA;
-    uint64_t *t_full = a_empty + SA, *t_empty = t_full + 2, *drain = t_empty + 2;
+    uint64_t *ready = bars, *consumed = ready + kTcSlots;
+    uint64_t *p_full = consumed + kTcSlots, *p_empty = p_full + SP;
+    uint64_t *t_full = p_empty + SP, *drain = t_full + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < SX; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
-        for (int i = 0; i < SP; ++i) { mbar_init(&p_full[i], 1); mbar_init(&p_empty[i], 4); }
-        for (int i = 0; i < SA; ++i) { mbar_init(&a_full[i], 4); mbar_init(&a_empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&t_full[i], 1); mbar_init(&t_empty[i], kTcPromoteWarps); }
+        // ready: x producer (1, plus transaction bytes) + 4 unpack warps + the promotion warps
+        for (int i = 0; i < kTcSlots; ++i) { mbar_init(&ready[i], 1 + 4 + kTcPromoteWarps); mbar_init(&consumed[i], 1); }
+        for (int i = 0; i < SP; ++i) { mbar_init(&p_full[i], 1); mbar_init(&p_empty[i], 4 * 32); }
+        for (int i = 0; i < 2; ++i) mbar_init(&t_full[i], 1);
         mbar_init(drain, 1);
         *abort = 0;
         fence_barrier_init();
@@ -242,28 +247,30 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         // ---------------------------------------------------------- x / t producer
         tma_prefetch_desc(&x_map);
         tma_prefetch_desc(&t_map);
-        int armed[SX];
-        for (int i = 0; i < SX; ++i) armed[i] = -1;
-        uint32_t s = 0, ph = 0;
+        int armed[kTcSlots];
+        for (int i = 0; i < kTcSlots; ++i) armed[i] = -1;
+        uint32_t unit = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int mt = tile % p.tiles_m;
-            for (int u = 0; u < U; ++u) {
+            for (int u = 0; u < U; ++u, ++unit) {
+                const uint32_t slot = unit % kTcSlots, ph = (unit / kTcSlots) & 1;
                 const int nst = (u < G) ? 2 : lowrank_stages(p.rank);
+                if (!mbar_wait(&consumed[slot], ph ^ 1, abort)) goto x_done;
+                mbar_arrive_expect_tx(&ready[slot], nst * L::kXBytes);
+                armed[slot] = (int)ph;
                 for (int st = 0; st < nst; ++st) {
-                    if (!mbar_wait(&x_empty[s], ph ^ 1, abort)) goto x_done;
-                    mbar_arrive_expect_tx(&x_full[s], L::kXBytes);
-                    armed[s] = (int)ph;
-                    uint8_t *dst = smem + L::kOffX + s * L::kXBytes;
-                    if (u < G) tma_load_2d(dst, &x_map, &x_full[s], (2 * u + st) * kTcBK, mt * kTcBT);
-                    else tma_load_2d(dst, &t_map, &x_full[s], st * kTcBK, mt * kTcBT);
-                    if (++s == SX) { s = 0; ph ^= 1; }
+                    uint8_t *dst = smem + L::kOffX + (slot * 2 + st) * L::kXBytes;
+                    if (u < G) tma_load_2d(dst, &x_map, &ready[slot], (2 * u + st) * kTcBK, mt * kTcBT);
+                    else tma_load_2d(dst, &t_map, &ready[slot], st * kTcBK, mt * kTcBT);
                 }
             }
         }
     x_done:
-        for (int i = 0; i < SX; ++i) {
+        // wait (bounded) for the copies still in flight: a slot's phase cannot complete without
+        // them, so poll the transaction count through the phase of the last armed unit
+        for (int i = 0; i < kTcSlots; ++i) {
             int local = 0;
-            if (armed[i] >= 0) (void)mbar_wait(&x_full[i], (uint32_t)armed[i], &local);
+            if (armed[i] >= 0 && *abort) (void)mbar_wait(&ready[i], (uint32_t)armed[i], &local, 50ull * 1000ull * 1000ull);
         }
     } else if (warp == 2 && lane == 0) {
         // ---------------------------------------------------------- packed-weight producer
@@ -289,30 +296,25 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
     } else if (warp == 1 && lane == 0) {
         // ---------------------------------------------------------- MMA issuer
         constexpr uint32_t idesc = umma_idesc_bf16(kTcBW, kTcBT);
-        uint32_t sa = 0, pa = 0, sx = 0, px = 0, unit = 0;
+        uint32_t unit = 0;
+        const uint32_t x_base = smem_u32(smem + L::kOffX);
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             for (int u = 0; u < U; ++u, ++unit) {
-                const uint32_t tb = unit & 1, tph = (unit >> 1) & 1;
-                if (!mbar_wait(&t_empty[tb], tph ^ 1, abort)) goto m_done;
+                const uint32_t slot = unit % kTcSlots, ph = (unit / kTcSlots) & 1, tb = unit & 1;
+                if (!mbar_wait(&ready[slot], ph, abort)) goto m_done;
                 tc_fence_after();
                 const uint32_t d = tmem + kTmemT0 + tb * kTcBT;
                 const int nst = (u < G) ? 2 : lowrank_stages(p.rank);
                 for (int st = 0; st < nst; ++st) {
                     const int nk = (u < G) ? kTcBK / 16 : min(kTcBK, 2 * p.rank - st * kTcBK) / 16;
-                    if (!mbar_wait(&a_full[sa], pa, abort)) goto m_done;
-                    if (!mbar_wait(&x_full[sx], px, abort)) goto m_done;
-                    tc_fence_after();
-                    const uint32_t a = tmem + kTmemA + sa * (kTcBK / 2);
-                    const uint32_t b_base = smem_u32(smem + L::kOffX + sx * L::kXBytes);
+                    const uint32_t a = tmem + kTmemA + (slot * 2 + st) * (kTcBK / 2);
+                    const uint32_t b_base = x_base + (slot * 2 + st) * L::kXBytes;
                     for (int k = 0; k < nk; ++k) {
                         const uint64_t bd = umma_desc_sw128(b_base + k * 32, 1024);
                         umma_bf16_ts(d, a + k * 8, bd, idesc, (st > 0 || k > 0) ? 1u : 0u);
                     }
-                    umma_commit(&a_empty[sa]);
-                    umma_commit(&x_empty[sx]);
-                    if (++sa == SA) { sa = 0; pa ^= 1; }
-                    if (++sx == SX) { sx = 0; px ^= 1; }
                 }
+                umma_commit(&consumed[slot]);
                 umma_commit(&t_full[tb]);
             }
         }
@@ -328,74 +330,67 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         const int quarter = warp & 3;
         const int row_local = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        uint32_t sa = 0, pa = 0, sp = 0, pp = 0;
+        uint32_t sp = 0, pp = 0, unit = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int nt = tile / p.tiles_m;
             const int64_t n = (int64_t)nt * kTcBW + row_local;
             const bool row_ok = n < p.N;
-            for (int g = 0; g < G; ++g) {
-                if (!warp_wait(&p_full[sp], pp, abort)) goto u_done;
-                uint32_t w[NWG];
-                {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(smem + L::kOffP + sp * L::kPBytes +
-                                                                        row_local * 16 * BITS);
+            for (int u = 0; u < U; ++u, ++unit) {
+                const uint32_t slot = unit % kTcSlots, ph = (unit / kTcSlots) & 1;
+                const uint32_t a_addr = tmem + lane_addr + kTmemA + slot * 2 * (kTcBK / 2);
+                if (u < G) {
+                    if (!warp_wait(&p_full[sp], pp, abort)) goto u_done;
+                    uint32_t w[NWG];
+                    {
+                        const uint4 *src = reinterpret_cast<const uint4 *>(smem + L::kOffP + sp * L::kPBytes +
+                                                                            row_local * 16 * BITS);
 #pragma unroll
-                    for (int i = 0; i < BITS; ++i) {
-                        const uint4 v = src[i];
-                        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-                    }
-                    w[4 * BITS] = 0;
-                }
-                const uint32_t sp_used = sp;
-                if (++sp == SP) { sp = 0; pp ^= 1; }
-                bool ok = true;
-                static_for<2>([&](auto hh) {
-                    constexpr int h = decltype(hh)::value;
-                    if (!ok) return;
-                    uint32_t q[32];
-                    unpack_half<BITS, h>(w, q);
-                    if (!warp_wait(&a_empty[sa], pa ^ 1, abort)) { ok = false; return; }
-                    tc_fence_after();        // order the store after the MMAs that read this stage
-                    tmem_st_32x32b_x32(tmem + lane_addr + kTmemA + sa * (kTcBK / 2), q);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&a_full[sa]);
-                    if (++sa == SA) { sa = 0; pa ^= 1; }
-                });
-                // the stage's bytes have been consumed by every lane (both halves are in TMEM):
-                // only now may the producer overwrite it
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&p_empty[sp_used]);
-                if (!ok) goto u_done;
-            }
-            if (p.rank > 0) {
-                // low-rank unit: A[n][k] = L2[k mod rank][n] for k < 2 rank (both halves of
-                // [t_hi | t_lo] meet the same L2), zero beyond
-                const int nst = lowrank_stages(p.rank);
-                for (int st = 0; st < nst; ++st) {
-                    uint32_t q[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int k = st * kTcBK + 2 * i;
-                        uint32_t v = 0;
-                        if (row_ok && k < 2 * p.rank) {
-                            const int j = k % p.rank;
-                            const uint32_t a = __ldg(p.L2 + (int64_t)j * p.N + n);
-                            const uint32_t b = __ldg(p.L2 + (int64_t)(j + 1) * p.N + n);
-                            v = a | (b << 16);
+                        for (int i = 0; i < BITS; ++i) {
+                            const uint4 v = src[i];
+                            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
                         }
-                        q[i] = v;
+                        w[4 * BITS] = 0;
                     }
-                    if (!warp_wait(&a_empty[sa], pa ^ 1, abort)) goto u_done;
+                    // every consuming thread releases the stage itself (arrival count 128): the
+                    // release then covers that thread's own shared-memory loads. A single arrive
+                    // after a warp sync does not: other lanes' loads may still be in flight when
+                    // the producer's next copy lands.
+                    mbar_arrive(&p_empty[sp]);
+                    if (++sp == SP) { sp = 0; pp ^= 1; }
+                    uint32_t q0[32], q1[32];
+                    unpack_half<BITS, 0>(w, q0);
+                    unpack_half<BITS, 1>(w, q1);
+                    if (!warp_wait(&consumed[slot], ph ^ 1, abort)) goto u_done;
+                    tc_fence_after();        // order the stores after the MMAs that read this slot
+                    tmem_st_32x32b_x32(a_addr, q0);
+                    tmem_st_32x32b_x32(a_addr + kTcBK / 2, q1);
+                } else {
+                    // low-rank unit: A[n][k] = L2[k mod rank][n] for k < 2 rank (both halves of
+                    // [t_hi | t_lo] meet the same L2), zero beyond
+                    if (!warp_wait(&consumed[slot], ph ^ 1, abort)) goto u_done;
                     tc_fence_after();
-                    tmem_st_32x32b_x32(tmem + lane_addr + kTmemA + sa * (kTcBK / 2), q);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&a_full[sa]);
-                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                    const int nst = lowrank_stages(p.rank);
+                    for (int st = 0; st < nst; ++st) {
+                        uint32_t q[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int k = st * kTcBK + 2 * i;
+                            uint32_t v = 0;
+                            if (row_ok && k < 2 * p.rank) {
+                                const int j = k % p.rank;
+                                const uint32_t a = __ldg(p.L2 + (int64_t)j * p.N + n);
+                                const uint32_t b = __ldg(p.L2 + (int64_t)(j + 1) * p.N + n);
+                                v = a | (b << 16);
+                            }
+                            q[i] = v;
+                        }
+                        tmem_st_32x32b_x32(a_addr + st * (kTcBK / 2), q);
+                    }
                 }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ready[slot]);
             }
         }
     u_done:;
@@ -406,6 +401,8 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         const int row_local = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         constexpr int kPre = 4;                                     // scale prefetch distance
+        // both T buffers start free: count this warp's release for units 0 and 1
+        if (lane == 0) { mbar_arrive(&ready[0]); mbar_arrive(&ready[1]); }
         uint32_t unit = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int mt = tile % p.tiles_m, nt = tile / p.tiles_m;
@@ -437,7 +434,7 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                         // both halves of T are in registers: hand the buffer back to the MMA
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&t_empty[tb]);
+                        if (lane == 0) mbar_arrive(&ready[(unit + 2) % kTcSlots]);
                     }
                     if (u == 0) {
 #pragma unroll
