@@ -19,8 +19,8 @@
 // 8 stages of codes (32 columns = 64 k each).
 // Warp roles (512 threads):
 //   warp 0      TMA producer of x tiles (128 tokens x 64 k bf16, 128B swizzle, 16 KB/stage)
-//   warp 1      TMEM allocator; one thread issues tcgen05.mma (A = codes from TMEM,
-//               B = x from shared memory, M=128 N=128 K=16) into T
+//   warps 1, 3  warp 1 allocates TMEM; one thread of each issues tcgen05.mma (A = codes from
+//               TMEM, B = x from shared memory, M=128 N=128 K=16) for alternate units
 //   warp 2      TMA producer of packed-weight tiles (128 rows x one group, 16*b bytes a row)
 //   warps 4-7   unpack: one weight row per thread; bf16 pairs of exact q written to the A
 //               stage with tcgen05.st
@@ -71,7 +71,7 @@ struct TcLayout {
     static constexpr uint32_t kOffX = 0;
     static constexpr uint32_t kOffP = kOffX + kTcStagesX * kXBytes;
     static constexpr uint32_t kOffBar = kOffP + kSP * kPBytes;
-    static constexpr uint32_t kNumBars = 2 * kTcSlots + 2 * kSP + 2 + 1;
+    static constexpr uint32_t kNumBars = 2 * kTcSlots + 2 * kSP + 2 + 2;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kBytes = kOffMisc + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;               // slack to align the base to 1024 B
@@ -216,7 +216,7 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
     uint64_t *ready = bars, *consumed = ready + kTcSlots;
     uint64_t *p_full = consumed + kTcSlots, *p_empty = p_full + SP;
-    uint64_t *t_full = p_empty + SP, *drain = t_full + 2;
+    uint64_t *t_full = p_empty + SP, *drain = t_full + 2;      // drain[2]: one per MMA thread
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
 
@@ -226,7 +226,8 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         for (int i = 0; i < kTcSlots; ++i) { mbar_init(&ready[i], 1 + 4 + kTcPromoteWarps); mbar_init(&consumed[i], 1); }
         for (int i = 0; i < SP; ++i) { mbar_init(&p_full[i], 1); mbar_init(&p_empty[i], 4 * 32); }
         for (int i = 0; i < 2; ++i) mbar_init(&t_full[i], 1);
-        mbar_init(drain, 1);
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
         *abort = 0;
         fence_barrier_init();
     }
@@ -293,13 +294,18 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
             int local = 0;
             if (armed[i] >= 0) (void)mbar_wait(&p_full[i], (uint32_t)armed[i], &local);
         }
-    } else if (warp == 1 && lane == 0) {
-        // ---------------------------------------------------------- MMA issuer
+    } else if ((warp == 1 || warp == 3) && lane == 0) {
+        // ---------------------------------------------------------- MMA issuers
+        // Two threads issue: warp 1 the even units (into T0), warp 3 the odd units (into T1).
+        // An MMA issue occupies the issuing thread for ~85 cycles and each unit also costs a
+        // barrier wait and two commits; a second issuer overlaps that with the other's MMAs.
+        const uint32_t mine = (warp == 1) ? 0u : 1u;
         constexpr uint32_t idesc = umma_idesc_bf16(kTcBW, kTcBT);
         uint32_t unit = 0;
         const uint32_t x_base = smem_u32(smem + L::kOffX);
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             for (int u = 0; u < U; ++u, ++unit) {
+                if ((unit & 1u) != mine) continue;
                 const uint32_t slot = unit % kTcSlots, ph = (unit / kTcSlots) & 1, tb = unit & 1;
                 if (!mbar_wait(&ready[slot], ph, abort)) goto m_done;
                 tc_fence_after();
@@ -321,9 +327,9 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
     m_done:
         {
             // every MMA issued by this thread completes before TMEM is released
-            umma_commit(drain);
+            umma_commit(&drain[mine]);
             int local = 0;
-            (void)mbar_wait(drain, 0, &local);
+            (void)mbar_wait(&drain[mine], 0, &local);
         }
     } else if (warp >= kTcUnpackWarp0 && warp < kTcPromoteWarp0) {
         // ---------------------------------------------------------- unpack codes into TMEM
@@ -351,10 +357,12 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                         }
                         w[4 * BITS] = 0;
                     }
-                    // every consuming thread releases the stage itself (arrival count 128): the
-                    // release then covers that thread's own shared-memory loads. A single arrive
-                    // after a warp sync does not: other lanes' loads may still be in flight when
-                    // the producer's next copy lands.
+                    // Every consuming thread releases the stage itself (arrival count 128), after a
+                    // proxy fence: its loads are generic-proxy reads and the producer's next copy
+                    // is an async-proxy write, so the reads are ordered before the release across
+                    // proxies. (One lane's arrive after a warp sync let the next copy land while
+                    // other lanes' loads were in flight.)
+                    fence_proxy_async_smem();
                     mbar_arrive(&p_empty[sp]);
                     if (++sp == SP) { sp = 0; pp ^= 1; }
                     uint32_t q0[32], q1[32];
