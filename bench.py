@@ -382,6 +382,71 @@ def e2e_leg(wq, lins, ws, args, device, world, step_flops):
             "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
+def case_arm(args):
+    """--case: time one call shape (for kernel timing and ncu captures).
+
+    pack:N,K,bits            quantize+pack of an N x K weight
+    linear:M,N,K,bits,rank   quantized linear (bias included), path from --path
+    Inputs are seeded torch draws on the GPU (weights ~N(0, 0.02^2), x ~N(0, 1)).
+    """
+    import torch
+    import bit_weight_quantization_wq_b200 as wq
+    from bit_weight_quantization_wq_b200 import build as wq_build
+    wq_build.build()
+    kind, _, spec = args.case.partition(":")
+    vals = [int(v) for v in spec.split(",")]
+    g = torch.Generator(device="cuda").manual_seed(1234)
+    dev = torch.device("cuda")
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    if kind == "pack":
+        N, K, bits = vals
+        W = (torch.randn(N, K, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+        packed = torch.empty((N, K * bits // 8), dtype=torch.uint8, device=dev)
+        scales = torch.empty((N, K // 128), dtype=torch.float32, device=dev)
+        run = lambda: wq.wq_quantize_pack(W, bits, packed=packed, scales=scales)
+        work = {"params": N * K, "bytes": 2 * N * K + N * K * bits / 8 + N * K / 32}
+    elif kind == "linear":
+        M, N, K, bits, rank = vals
+        W = (torch.randn(N, K, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+        x = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
+        b = (torch.randn(N, device=dev, generator=g) * 0.01).to(torch.bfloat16)
+        L1 = L2 = None
+        if rank:
+            L1 = (torch.randn(K, rank, device=dev, generator=g) * 0.05).to(torch.bfloat16)
+            L2 = (torch.randn(rank, N, device=dev, generator=g) * 0.05).to(torch.bfloat16)
+        packed, scales = wq.wq_quantize_pack(W, bits)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(16, wq.wq_linear_workspace_bytes(M, N, K, bits, rank)), dtype=torch.uint8, device=dev)
+        run = lambda: wq.wq_linear(x, packed, scales, bits, N, L1=L1, L2=L2, bias=b, y=y, workspace=ws, path=args.path)
+        work = {"flops": gemm_flops(N, K, M, rank), "weight_bytes": weight_bytes(N, K, bits),
+                "bytes": 2 * M * K + 2 * M * N + weight_bytes(N, K, bits) + 2 * rank * (K + N) + 2 * N}
+    else:
+        raise SystemExit(f"unknown case kind {kind!r}")
+    for _ in range(max(3, args.warmup)):
+        run()
+    torch.cuda.synchronize()
+    ev[0].record()
+    for _ in range(args.steps):
+        run()
+    ev[1].record()
+    torch.cuda.synchronize()
+    us = ev[0].elapsed_time(ev[1]) / args.steps * 1e3
+    out = {"case": args.case, "path": args.path, "us_per_call": us, "status": wq.wq_device_status()}
+    peaks, src = load_peaks()
+    if "flops" in work:
+        out["tflops"] = work["flops"] / us / 1e6
+        out["weight_gbs"] = work["weight_bytes"] / us / 1e3
+        out["frac_bf16"] = out["tflops"] / peaks["bf16_tflops"]
+        out["frac_hbm"] = work["bytes"] / us / 1e3 / peaks["hbm_gbs"]
+    else:
+        out["gparams"] = work["params"] / us / 1e3
+        out["gbs"] = work["bytes"] / us / 1e3
+        out["frac_hbm"] = out["gbs"] / peaks["hbm_gbs"]
+    out["peak_source"] = src
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def parse(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -391,6 +456,8 @@ def parse(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--case", default=None, help="time one shape: pack:N,K,bits or linear:M,N,K,bits,rank")
+    ap.add_argument("--path", default="auto", choices=["auto", "small_m", "tensor"], help="kernel family for --case linear")
     return ap.parse_args(argv)
 
 
@@ -400,6 +467,8 @@ def main(argv=None):
         args.warmup = 3
     if args.impl == "reference":
         return reference_arm(args)
+    if args.case:
+        return case_arm(args)
     return main_arm(args)
 
 
