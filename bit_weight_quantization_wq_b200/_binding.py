@@ -30,6 +30,7 @@ SYMBOLS = (
     "wq_version", "wq_packed_bytes", "wq_scales_count", "wq_quantize_pack",
     "wq_linear_workspace_bytes", "wq_linear", "wq_linear_ex", "wq_device_status",
     "wq_selftest_bounded_wait", "wq_status_string", "wq_last_error", "wq_launch_count",
+    "wq_linear_no_workspace",
 )
 
 
@@ -72,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.wq_status_string.argtypes, L.wq_status_string.restype = [i32], ctypes.c_char_p
         L.wq_last_error.argtypes, L.wq_last_error.restype = [], ctypes.c_char_p
         L.wq_launch_count.argtypes, L.wq_launch_count.restype = [], ctypes.c_uint64
+        L.wq_linear_no_workspace.argtypes = [p, i64, i64, p, p, i32, i32, i64, p, p, i32, p, p, p]
+        L.wq_linear_no_workspace.restype = i32
         _lib = L
     return _lib
 

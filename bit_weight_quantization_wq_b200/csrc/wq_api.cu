@@ -285,6 +285,26 @@ wq_status tc_linear(const TcArgs &a, int sm_count, cudaStream_t st) {
 
 size_t smallm_workspace(int64_t M, int rank) { return rank > 0 ? align_up((size_t)M * rank * 4, 256) : 0; }
 
+// ------------------------------------------------------------------ static scratch
+// Scratch for wq_linear_no_workspace: a file-scope device array. In host code its name is
+// only a stand-in, so the kernels get the address cudaGetSymbolAddress reports, looked up
+// once per device with that device current.
+static __device__ __align__(256) unsigned char g_static_scratch[WQ_STATIC_SCRATCH_BYTES];
+void *g_static_scratch_ptr[kMaxDevices] = {};
+std::mutex g_static_scratch_mutex;
+
+wq_status static_scratch(int dev, void **out) {
+    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+    if (!g_static_scratch_ptr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+        g_static_scratch_ptr[dev] = p;
+    }
+    *out = g_static_scratch_ptr[dev];
+    return WQ_OK;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -420,6 +440,29 @@ wq_status wq_linear(const void *x, int64_t M, int64_t K, const uint8_t *packed, 
                     void *workspace, size_t workspace_bytes, wq_stream_t stream) {
     return wq_linear_ex(x, M, K, packed, scales, bits, group, N, L1, L2, rank, bias, y, workspace,
                         workspace_bytes, WQ_PATH_AUTO, stream);
+}
+
+wq_status wq_linear_no_workspace(const void *x, int64_t M, int64_t K, const uint8_t *packed, const float *scales,
+                                 int bits, int group, int64_t N, const void *L1, const void *L2, int rank,
+                                 const void *bias, void *y, wq_stream_t stream) {
+    g_last_error[0] = 0;
+    const size_t need = wq_linear_workspace_bytes(M, N, K, bits, rank);
+    if (need > WQ_STATIC_SCRATCH_BYTES)
+        return fail(WQ_ERR_WORKSPACE, "scratch of %zu bytes needed, the static buffer holds %zu", need,
+                    (size_t)WQ_STATIC_SCRATCH_BYTES);
+    void *scratch = nullptr;
+    size_t scratch_bytes = 0;
+    if (need > 0) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+        if (dev < 0 || dev >= kMaxDevices) return fail(WQ_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
+        wq_status s = static_scratch(dev, &scratch);
+        if (s != WQ_OK) return s;
+        scratch_bytes = WQ_STATIC_SCRATCH_BYTES;
+    }
+    return wq_linear_ex(x, M, K, packed, scales, bits, group, N, L1, L2, rank, bias, y, scratch, scratch_bytes,
+                        WQ_PATH_AUTO, stream);
 }
 
 wq_status wq_device_status(wq_stream_t stream, int clear) {

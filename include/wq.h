@@ -119,6 +119,30 @@ WQ_API wq_status wq_linear(const void *x, int64_t M, int64_t K,
                     const void *L1, const void *L2, int rank, const void *bias,
                     void *y, void *workspace, size_t workspace_bytes, wq_stream_t stream);
 
+/*
+ * wq_linear without a caller-provided workspace. There is no counterpart of this call on
+ * the pages; it exists for callers that cannot allocate device memory when they run the
+ * layer -- for example code that owns no allocator (a plugin handed raw tensors by a host
+ * framework), code running under a fixed device-memory budget that has already been handed
+ * out, or a real-time loop in which an allocation could block or fail.
+ * The low-rank branch needs scratch; this call uses a buffer of WQ_STATIC_SCRATCH_BYTES that
+ * is compiled into the library (every GPU that loads libwq.so holds it until the process
+ * exits). Sizes whose scratch would exceed it -- wq_linear_workspace_bytes(M, N, K, bits,
+ * rank) > WQ_STATIC_SCRATCH_BYTES, e.g. more than 16384 tokens with a low-rank branch --
+ * are rejected with WQ_ERR_WORKSPACE before anything is launched; calls without the branch
+ * never touch it. The call allocates nothing and frees nothing.
+ * The first call on a device looks up the buffer's device address once (with that device
+ * current); make that first call before any stream capture. Every call on a device shares
+ * the one buffer, and it keeps the last call's contents: calls whose work overlaps on the
+ * GPU (different streams, no ordering between them) race on it. Arguments and results are
+ * otherwise exactly those of wq_linear.
+ */
+#define WQ_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
+WQ_API wq_status wq_linear_no_workspace(const void *x, int64_t M, int64_t K,
+                                        const uint8_t *packed, const float *scales, int bits, int group,
+                                        int64_t N, const void *L1, const void *L2, int rank,
+                                        const void *bias, void *y, wq_stream_t stream);
+
 /* wq_linear with an explicit kernel family (for tests and benchmarks). */
 WQ_API wq_status wq_linear_ex(const void *x, int64_t M, int64_t K,
                        const uint8_t *packed, const float *scales, int bits, int group, int64_t N,

@@ -29,7 +29,7 @@ def header_functions():
 
 def test_exports_match_header(L):
     declared = header_functions()
-    assert len(declared) == 12
+    assert len(declared) == 13
     out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
     exported = sorted(line.split()[-1] for line in out.splitlines() if line.split()[-1].startswith("wq_"))
