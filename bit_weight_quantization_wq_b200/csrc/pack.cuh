@@ -7,8 +7,22 @@
 //
 // Layout: the W rows are contiguous 128-element groups, so group G = n * (K/128) + g sits
 // at bf16 offset 128 G, its packed bytes at 16*b*G and its scale at G. The kernel is a flat
-// grid-stride loop over groups: a half-warp owns one group, each lane 8 weights (one 16-byte
-// load) and therefore exactly b output bytes.
+// grid-stride loop over groups: four lanes own one group, each lane 32 consecutive weights
+// (64 bytes) and therefore exactly 4*b output bytes (b whole words).
+//
+// The kernel is HBM-bound only if it stays under ~8 instructions per weight, so every step
+// is chosen for its instruction count:
+//   * abs_max: bf16x2 max of magnitudes (max.xorsign.abs) over the lane's 16 words, then
+//     two shuffles across the group's four lanes;
+//   * step = RN(2s / (2^b - 1)) by one-correction division with the correctly rounded
+//     constant y = RN(1/L): q0 = RN(2s y), r = 2s - L q0 (exact by fma),
+//     step = RN(q0 + r y). This is Markstein's correction step; it was checked to equal the
+//     IEEE quotient for every bf16 abs_max whose 2s lies in [2^-120, 2^120] and every L in
+//     {7, 15, 31, 63, 127}. Outside that range the kernel divides.
+//   * quantize two weights per instruction with the packed fp32 pair operations of sm_100
+//     (mul/add/sub .f32x2);
+//   * codes are formed by the fp32 adder itself (see "Codes" below) and packed with shifts,
+//     byte permutes and one 16-byte (4-bit) or b 4-byte stores.
 //
 // Exactness: q must equal round_half_even(fl32(w / step)). The kernel multiplies by the
 // correctly rounded reciprocal and recomputes with an IEEE division only when the product
@@ -16,8 +30,20 @@
 // r' = RN(w * inv) = (w/step)(1 + d1)(1 + d2), |d1|, |d2| <= 2^-24, while
 // RN(w / step) = (w/step)(1 + d3). For |w/step| < 64 (always true, b <= 7) the two differ
 // by less than 64 * 3 * 2^-24 < 1.2e-5, so outside the 4e-5 window both round to the same
-// integer. Rounding to the nearest integer uses the 1.5 * 2^23 magic constant (an fp32 add
-// rounds to nearest even at that magnitude), valid for |r| < 2^22.
+// integer.
+//
+// Codes: for a weight pair (a, b) = elements (2i, 2i+1), t_a = RN(r_a + 1.5 * 2^23) and
+// t_b = RN(r_b + 2^23 + o (2^b + 1)), o = 2^(b-1). Both constants are even and both sums lie
+// in [2^23, 2^24), where fp32 spacing is 1, so each add rounds r to the nearest integer with
+// ties to even: t_a = 1.5 * 2^23 + q_a, t_b = 2^23 + o (2^b + 1) + q_b exactly. Then
+// fma(t_a - 1.5 * 2^23, 2^b, t_b) = 2^23 + (q_a + o) 2^b + (q_b + o) is exact, so the low 2b
+// mantissa bits of that float are the two codes, first code high: the pair field of the
+// MSB-first bitstream.
+//
+// Clamp: the page clamps q to +-(2^(b-1) - 1). The clamp never binds: |w| <= abs_max and
+// abs_max / step <= (2^b - 1) / 2.02 (1 + 2^-22) < 2^(b-1) - 1/2 for b = 3..7, so |q| <=
+// 2^(b-1) - 1 always (checked for every bf16 abs_max on the CPU). The kernel therefore has
+// no clamp. Weights must be finite; a group holding inf or NaN gets unspecified codes.
 #pragma once
 
 #include "common.cuh"
@@ -25,85 +51,168 @@
 namespace wq {
 
 constexpr int kPackThreads = 256;
-constexpr int kPackUnroll = 4;          // group pairs per warp per loop iteration
+constexpr int kPackUnroll = 2;          // 8-group blocks per warp per loop iteration
+constexpr int kPackGroupsPerWarp = 8 * kPackUnroll;
+
+__device__ __forceinline__ uint32_t bf16x2_maxabs(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+    return (uint64_t)__float_as_uint(a) | ((uint64_t)__float_as_uint(b) << 32);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
 
 template <int BITS>
 __global__ void __launch_bounds__(kPackThreads)
 quantize_pack_kernel(const uint16_t *__restrict__ W, int64_t n_groups,
                      uint8_t *__restrict__ packed, float *__restrict__ scales) {
     constexpr int kLevels = (1 << BITS) - 1;
-    constexpr int kQmax = kLevels / 2;
-    constexpr int kOffset = 1 << (BITS - 1);
+    constexpr int kOff = 1 << (BITS - 1);
     constexpr int kGroupBytes = 16 * BITS;
     constexpr int U = kPackUnroll;
-    constexpr int kWarpBytes = 2 * U * kGroupBytes;
-    constexpr float kMagic = 12582912.0f;               // 1.5 * 2^23
-    constexpr int kMagicBits = 0x4B400000;
-    __shared__ __align__(16) uint8_t stage[kPackThreads / 32][kWarpBytes];
+    constexpr int GW = kPackGroupsPerWarp;
+    constexpr float kL = (float)kLevels;
+    constexpr float kInvL = 1.0f / (float)kLevels;                  // RN(1/L), folded by the compiler
+    constexpr float kMagicA = 12582912.0f;                          // 1.5 * 2^23
+    constexpr float kMagicB = 8388608.0f + (float)(kOff * ((1 << BITS) + 1));
+    constexpr float kPow = (float)(1 << BITS);
+    constexpr uint32_t kMask2 = (1u << (2 * BITS)) - 1u;
+    constexpr int kStageWords = (BITS == 4) ? 1 : GW * 4 * BITS;
+    __shared__ __align__(16) uint32_t stage[kPackThreads / 32][kStageWords];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int half = lane >> 4, l16 = lane & 15;
-    uint8_t *st = stage[warp];
+    const int gi = lane >> 2, l4 = lane & 3;
     const int64_t warp_id = (int64_t)blockIdx.x * (kPackThreads / 32) + warp;
     const int64_t n_warps = (int64_t)gridDim.x * (kPackThreads / 32);
 
-    for (int64_t g0 = warp_id * 2 * U; g0 < n_groups; g0 += n_warps * 2 * U) {
-        uint4 v[U];
+    for (int64_t g0 = warp_id * GW; g0 < n_groups; g0 += n_warps * GW) {
+        uint32_t w[U][16];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t g = g0 + 2 * u + half;
-            v[u] = (g < n_groups) ? ldg_stream_v4(W + g * 128 + l16 * 8) : make_uint4(0, 0, 0, 0);
+            const int64_t g = g0 + 8 * u + gi;
+            const uint16_t *src = W + g * 128 + l4 * 32;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 v = (g < n_groups) ? ldg_nc_v4(src + 8 * i) : make_uint4(0, 0, 0, 0);
+                w[u][4 * i] = v.x; w[u][4 * i + 1] = v.y; w[u][4 * i + 2] = v.z; w[u][4 * i + 3] = v.w;
+            }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t g = g0 + 2 * u + half;
-            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-            // abs_max of the group: bf16 magnitudes compare like 15-bit integers
-            uint32_t m = 0;
+            const int64_t g = g0 + 8 * u + gi;
+            // ---- abs_max of the group (bf16 magnitudes; the max tree keeps only |.|)
+            uint32_t m8[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+            for (int i = 0; i < 8; ++i) m8[i] = bf16x2_maxabs(w[u][2 * i], w[u][2 * i + 1]);
 #pragma unroll
-            for (int off = 8; off >= 1; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+            for (int i = 0; i < 4; ++i) m8[i] = bf16x2_maxabs(m8[i], m8[i + 4]);
+            m8[0] = bf16x2_maxabs(m8[0], m8[2]);
+            m8[1] = bf16x2_maxabs(m8[1], m8[3]);
+            const uint32_t m2 = bf16x2_maxabs(m8[0], m8[1]) & 0x7FFF7FFFu;
+            uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+            m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
             const float abs_max = __uint_as_float(m << 16);
-            const float s = __fmul_rn(abs_max, 1.01f);
-            const float step = __fdiv_rn(__fmul_rn(2.0f, s), (float)kLevels);
-            const bool zero = (step == 0.0f);
-            float inv = zero ? 0.0f : __frcp_rn(step);
-            const bool slow = !(inv <= 3.402823466e38f);    // 1/step overflowed: divide always
-            if (slow) inv = 0.0f;
-
-            uint64_t stream = 0;                            // 8 codes, first code highest
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t h = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
-                const float x = __uint_as_float(h << 16);
-                float r = __fmul_rn(x, inv);
-                float t = __fadd_rn(r, kMagic);
-                const float e = __fsub_rn(r, __fadd_rn(t, -kMagic));
-                if (slow || fabsf(e) > 0.49996f) {
-                    r = __fdiv_rn(x, step);
-                    t = __fadd_rn(r, kMagic);
-                }
-                int q = __float_as_int(t) - kMagicBits;
-                q = min(max(q, -kQmax), kQmax);
-                stream = (stream << BITS) | (uint32_t)(q + kOffset);
-            }
-            // this lane's BITS bytes, most significant first, at its place in the group
-            uint8_t *dst = st + (2 * u + half) * kGroupBytes + l16 * BITS;
-            if constexpr (BITS == 4) {
-                *reinterpret_cast<uint32_t *>(dst) = __byte_perm((uint32_t)stream, 0, 0x0123);
+            // ---- step = RN(2 s / L), s = RN(abs_max * 1.01)
+            const float two = __fmul_rn(2.0f, __fmul_rn(abs_max, 1.01f));
+            float step;
+            if (two >= 7.52316384526264e-37f && two <= 1.329227995784916e36f) {   // [2^-120, 2^120]
+                const float q0 = __fmul_rn(two, kInvL);
+                const float r = __fmaf_rn(-q0, kL, two);
+                step = __fmaf_rn(r, kInvL, q0);
             } else {
-#pragma unroll
-                for (int j = 0; j < BITS; ++j) dst[j] = (uint8_t)(stream >> (8 * (BITS - 1 - j)));
+                step = __fdiv_rn(two, kL);
             }
-            if (l16 == 0 && g < n_groups) scales[g] = step;
+            float inv = (step == 0.0f) ? 0.0f : __frcp_rn(step);
+            bool near = !(inv <= 3.402823466e38f);           // 1/step overflowed: divide always
+            if (near) inv = 0.0f;
+            // ---- quantize, two weights per instruction
+            const uint64_t inv2 = f2(inv, inv), magic = f2(kMagicA, kMagicB);
+            // pair fields: the low 2b bits of F[i] = code(2i) << b | code(2i+1)
+            uint32_t F[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint64_t x2 = (uint64_t)(w[u][i] << 16) | ((uint64_t)(w[u][i] & 0xFFFF0000u) << 32);
+                const uint64_t r2 = mul2(x2, inv2);
+                const uint64_t t2 = add2(r2, magic);
+                const uint64_t q2 = sub2(t2, magic);
+                const uint64_t e2 = sub2(r2, q2);
+                near |= (fabsf(f2_lo(e2)) > 0.49996f) | (fabsf(f2_hi(e2)) > 0.49996f);
+                F[i] = __float_as_uint(__fmaf_rn(f2_lo(q2), kPow, f2_hi(t2)));
+            }
+            if (near) {
+                // rare: a product close to a half-integer (or a huge 1/step): IEEE division
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float xa = __uint_as_float(w[u][i] << 16), xb = __uint_as_float(w[u][i] & 0xFFFF0000u);
+                    const float ra = (step == 0.0f) ? 0.0f : __fdiv_rn(xa, step);
+                    const float rb = (step == 0.0f) ? 0.0f : __fdiv_rn(xb, step);
+                    const float qa = __fsub_rn(__fadd_rn(ra, kMagicA), kMagicA);
+                    F[i] = __float_as_uint(__fmaf_rn(qa, kPow, __fadd_rn(rb, kMagicB)));
+                }
+            }
+            if (l4 == 0 && g < n_groups) scales[g] = step;
+            if constexpr (BITS == 4) {
+                // a pair field is one whole byte (bits 8..22 of the float are zero)
+                uint32_t o[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    o[k] = __byte_perm(__byte_perm(F[4 * k], F[4 * k + 1], 0x0040u),
+                                       __byte_perm(F[4 * k + 2], F[4 * k + 3], 0x0040u), 0x5410u);
+                if (g < n_groups)
+                    *reinterpret_cast<uint4 *>(packed + g * kGroupBytes + l4 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+            } else {
+                // quad fields (4 codes, 4b bits), placed into the 32b-bit stream number whose
+                // most significant bits hold the first code; memory order is big-endian
+                uint32_t Nw[BITS];
+#pragma unroll
+                for (int k = 0; k < BITS; ++k) Nw[k] = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t T = ((F[2 * j] & kMask2) << (2 * BITS)) | (F[2 * j + 1] & kMask2);
+                    const int o = 4 * BITS * (7 - j), wd = o / 32, sh = o % 32;
+                    Nw[wd] |= T << sh;
+                    if (sh + 4 * BITS > 32) Nw[wd + 1] |= T >> (32 - sh);
+                }
+                uint32_t *dst = stage[warp] + (8 * u + gi) * 4 * BITS + l4 * BITS;
+#pragma unroll
+                for (int k = 0; k < BITS; ++k) dst[k] = __byte_perm(Nw[BITS - 1 - k], 0, 0x0123u);
+            }
         }
-        __syncwarp();
-        const int64_t valid = min((int64_t)(2 * U), n_groups - g0);
-        const int chunks = (int)(valid * kGroupBytes / 16);
-        uint4 *out = reinterpret_cast<uint4 *>(packed + g0 * kGroupBytes);
-        for (int c = lane; c < chunks; c += 32) out[c] = reinterpret_cast<const uint4 *>(st)[c];
-        __syncwarp();
+        if constexpr (BITS != 4) {
+            __syncwarp();
+            const int64_t valid = min((int64_t)GW, n_groups - g0);
+            const int chunks = (int)(valid * kGroupBytes / 16);
+            uint4 *out = reinterpret_cast<uint4 *>(packed + g0 * kGroupBytes);
+            for (int c = lane; c < chunks; c += 32) out[c] = reinterpret_cast<const uint4 *>(stage[warp])[c];
+            __syncwarp();
+        }
     }
 }
 

@@ -84,7 +84,7 @@ wq_status check_launch(const char *what) {
 template <int BITS>
 wq_status launch_pack(const void *W, int64_t n_groups, uint8_t *packed, float *scales, int sm_count,
                       cudaStream_t st) {
-    const int64_t per_block = 2 * wq::kPackUnroll * (wq::kPackThreads / 32);
+    const int64_t per_block = (int64_t)wq::kPackGroupsPerWarp * (wq::kPackThreads / 32);
     const int64_t want = (n_groups + per_block - 1) / per_block;
     const int grid = (int)std::min<int64_t>(want, (int64_t)sm_count * 8);
     wq::quantize_pack_kernel<BITS><<<grid, wq::kPackThreads, 0, st>>>(

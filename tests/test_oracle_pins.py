@@ -235,6 +235,27 @@ def test_error_bound_and_code_range(bits):
 
 
 @pytest.mark.parametrize("bits", BITS)
+def test_clamp_never_binds_for_any_bf16_abs_max(bits):
+    """Sec. 3.1 clamps q to +-(2^(b-1) - 1). For every finite bf16 abs_max, the largest
+    quotient of the group, RN(abs_max / step) with the page's fp32 step, stays below
+    2^(b-1) - 1/2, so round() never reaches the clamp (|w| <= abs_max and RN is monotone).
+    numpy's float32 multiply and divide are IEEE correctly rounded."""
+    a = synth.bf16_bits_to_f32(np.arange(1, 0x7F80, dtype=np.uint16))
+    with np.errstate(over="ignore"):
+        s = a * np.float32(1.01)
+        step = (np.float32(2.0) * s) / np.float32((1 << bits) - 1)
+        r = a / step
+    assert np.isfinite(a).all() and r.dtype == np.float32
+    assert np.nanmax(r) < (1 << (bits - 1)) - 0.5
+    # and the oracle agrees: groups whose abs_max is each of these values keep codes in range
+    W = np.zeros((len(a) // 8, 128), np.uint16)
+    W[:, 0] = np.arange(1, 0x7F80, dtype=np.uint16)[: len(W) * 8 : 8]
+    W[:, 1] = W[:, 0] | 0x8000
+    codes, _ = oracle.quantize(W, bits)
+    assert codes.min() >= 1 and codes.max() <= (1 << bits) - 1
+
+
+@pytest.mark.parametrize("bits", BITS)
 def test_all_zero_group(bits):
     W = np.zeros((2, 256), np.uint16)
     W[1, 128:] = bf16(np.linspace(-1, 1, 128))

@@ -46,6 +46,22 @@ def test_pack_parity_edges(bits, N, K):
 
 
 @pytest.mark.parametrize("bits", BITS)
+def test_pack_parity_every_bf16_abs_max(bits):
+    """One group per finite positive bf16 value (0x0001 .. 0x7F7F, subnormals and the
+    values whose 2 * 1.01 * abs_max overflows fp32 included), that value as the group's
+    abs_max and the other weights below it: every step the kernel can produce, bit-exact."""
+    rng = np.random.default_rng(4242 + bits)
+    a_bits = np.arange(1, 0x7F80, dtype=np.uint16)
+    a = synth.bf16_bits_to_f32(a_bits).astype(np.float64)
+    u = rng.uniform(-1.0, 1.0, size=(len(a), 128))
+    W = synth.f32_to_bf16_bits((a[:, None] * u).astype(np.float32))
+    W[:, 0] = a_bits
+    W[1::2, 0] |= 0x8000                       # negative abs_max element on odd groups
+    W = W[: len(W) // 8 * 8].reshape(-1, 8 * 128)
+    _pack_check(W, bits)
+
+
+@pytest.mark.parametrize("bits", BITS)
 def test_pack_empty(bits):
     import torch
     W = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
