@@ -426,12 +426,12 @@ def case_arm(args):
     # that buffer (no write-back of dirty lines lands inside the timed call). The flush also
     # keeps the GPU busy while the host queues the call, so host overhead stays out of the
     # events.
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.empty(32 << 20, dtype=torch.int64, device=dev)      # 256 MB
     sink = torch.empty((), dtype=torch.int64, device=dev)
 
     def flush_l2():
         flush.fill_(1)
-        torch.sum(flush, dtype=torch.int64, out=sink)
+        torch.sum(flush, dim=0, out=sink)
 
     for _ in range(max(3, args.warmup)):
         flush_l2()

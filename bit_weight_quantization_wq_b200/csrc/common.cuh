@@ -105,6 +105,38 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// Order this thread's earlier generic-proxy shared-memory accesses before later async-proxy
+// (bulk copy / TMA) writes that another thread issues after a barrier handshake.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// All 32 lanes wait on a barrier phase; the give-up decision is taken by lane 0 so that the
+// warp leaves together.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    const int lane = threadIdx.x & 31;
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        const bool ok = mbar_try_wait(bar, parity);
+        if (__all_sync(0xffffffffu, ok)) return true;
+        if ((it & 63u) == 63u) {
+            int stop = 0;
+            if (lane == 0) {
+                const uint64_t now = globaltimer_ns();
+                if (t0 == 0) t0 = now;
+                if (*abort) {
+                    stop = 1;
+                } else if (now - t0 > kWaitLimitNs) {
+                    record_status(WQ_ERR_TIMEOUT);
+                    *abort = 1;
+                    stop = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+        }
+    }
+}
+
 // ------------------------------------------------------------------ TMA
 // 2D tiled bulk-tensor load into shared memory, completion on an mbarrier.
 // x is the innermost coordinate; x * element size must be a multiple of 16 bytes.
@@ -114,6 +146,15 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, ui
         "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];"
         ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+// 3D tiled bulk-tensor load (coordinates innermost first), completion on an mbarrier.
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, uint64_t *bar,
+                                            int32_t x, int32_t y, int32_t z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {

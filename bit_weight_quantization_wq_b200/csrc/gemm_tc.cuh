@@ -43,7 +43,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
-#include "smallm.cuh"
+#include "unpack.cuh"
 
 namespace wq {
 
@@ -89,119 +89,6 @@ struct TcParams {
 
 // k stages (64 wide) of the low-rank unit: [t_hi | t_lo] has 2 * rank columns.
 __host__ __device__ constexpr int lowrank_stages(int rank) { return (2 * rank + kTcBK - 1) / kTcBK; }
-
-template <int I> struct Int { static constexpr int value = I; };
-template <int N, int I = 0, class F>
-__device__ __forceinline__ void static_for(F &&f) {
-    if constexpr (I < N) {
-        f(Int<I>{});
-        static_for<N, I + 1>(f);
-    }
-}
-
-// Big-endian 8-code block BLK (b bytes at byte offset BLK*b) of a group held as words.
-template <int BITS, int BLK, int NW>
-__device__ __forceinline__ void tc_block_be(const uint32_t (&w)[NW], uint32_t &lo, uint32_t &hi) {
-    constexpr int o = BLK * BITS;
-    if constexpr (BITS == 3) {
-        lo = be32<o, NW>(w) >> 8;
-        hi = 0;
-    } else if constexpr (BITS == 4) {
-        lo = be32<o, NW>(w);
-        hi = 0;
-    } else {
-        lo = be32<o + BITS - 4, NW>(w);
-        hi = be32<o, NW>(w) >> (8 * (8 - BITS));
-    }
-}
-
-// PTX prmt in its default mode: selector nibble bits 2:0 pick one of the 8 source bytes and
-// bit 3 replaces it by copies of that byte's sign bit (zero for bytes below 0x80). The CUDA
-// __byte_perm intrinsic ignores bit 3, hence the inline form.
-__device__ __forceinline__ uint32_t prmt_sx(uint32_t a, uint32_t b, uint32_t sel) {
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-    return d;
-}
-
-// 32 bf16x2 words of exact q = code - 2^(b-1), in natural k order (word i = k 2i, 2i+1),
-// for codes [64 h, 64 h + 64) of a group held as 4*b little-endian words.
-template <int BITS, int H, int NW>
-__device__ __forceinline__ void unpack_half(const uint32_t (&w)[NW], uint32_t (&out)[32]) {
-    constexpr uint32_t kOff = 0x43004300u;                          // bf16 128 in each half
-    const __nv_bfloat162 corr = __floats2bfloat162_rn(128.0f + (1 << (BITS - 1)), 128.0f + (1 << (BITS - 1)));
-    if constexpr (BITS == 4) {
-        // byte j of a word = (code 2j << 4) | code 2j+1
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t v = w[8 * H + i];
-            const uint32_t hiN = (v >> 4) & 0x0F0F0F0Fu, loN = v & 0x0F0F0F0Fu;
-            // (hi nibble of byte j) | (lo nibble of byte j) << 16; the sign-replicating
-            // selector nibbles (8 + byte) give the zero high bytes
-            const uint32_t p0 = prmt_sx(hiN, loN, 0xC480u) + kOff;
-            const uint32_t p1 = prmt_sx(hiN, loN, 0xD591u) + kOff;
-            const uint32_t p2 = prmt_sx(hiN, loN, 0xE6A2u) + kOff;
-            const uint32_t p3 = prmt_sx(hiN, loN, 0xF7B3u) + kOff;
-            const uint32_t pp[4] = {p0, p1, p2, p3};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                __nv_bfloat162 t = *reinterpret_cast<const __nv_bfloat162 *>(&pp[j]);
-                t = __hsub2(t, corr);
-                out[4 * i + j] = *reinterpret_cast<uint32_t *>(&t);
-            }
-        }
-    } else {
-        constexpr uint32_t m = (1u << BITS) - 1u;
-        static_for<8>([&](auto bb) {
-            constexpr int blk = decltype(bb)::value;
-            uint32_t lo, hi;
-            tc_block_be<BITS, 8 * H + blk>(w, lo, hi);
-            static_for<4>([&](auto pp) {
-                constexpr int pr = decltype(pp)::value;
-                constexpr int sh = 2 * BITS * (3 - pr);
-                uint32_t G;
-                if constexpr (sh >= 32) G = hi >> (sh - 32);
-                else if constexpr (sh == 0) G = lo;
-                else G = __funnelshift_r(lo, hi, sh);
-                // G bits [0,b) = code 2pr+1, [b,2b) = code 2pr: low half <- G >> b, high half <- G
-                uint32_t r = (__byte_perm(G >> BITS, G, 0x5410u) & (m | (m << 16))) | kOff;
-                __nv_bfloat162 t = *reinterpret_cast<const __nv_bfloat162 *>(&r);
-                t = __hsub2(t, corr);
-                out[4 * blk + pr] = *reinterpret_cast<uint32_t *>(&t);
-            });
-        });
-    }
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// All 32 lanes wait on a barrier phase; the give-up decision is taken by lane 0 so that the
-// warp leaves together.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
-    const int lane = threadIdx.x & 31;
-    uint64_t t0 = 0;
-    for (uint32_t it = 0;; ++it) {
-        const bool ok = mbar_try_wait(bar, parity);
-        if (__all_sync(0xffffffffu, ok)) return true;
-        if ((it & 63u) == 63u) {
-            int stop = 0;
-            if (lane == 0) {
-                const uint64_t now = globaltimer_ns();
-                if (t0 == 0) t0 = now;
-                if (*abort) {
-                    stop = 1;
-                } else if (now - t0 > kWaitLimitNs) {
-                    record_status(WQ_ERR_TIMEOUT);
-                    *abort = 1;
-                    stop = 1;
-                }
-            }
-            if (__shfl_sync(0xffffffffu, stop, 0)) return false;
-        }
-    }
-}
 
 template <int BITS>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -366,8 +253,8 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                     mbar_arrive(&p_empty[sp]);
                     if (++sp == SP) { sp = 0; pp ^= 1; }
                     uint32_t q0[32], q1[32];
-                    unpack_half<BITS, 0>(w, q0);
-                    unpack_half<BITS, 1>(w, q1);
+                    unpack_pairs<BITS, 0, 8>(w, q0);
+                    unpack_pairs<BITS, 8, 8>(w, q1);
                     if (!warp_wait(&consumed[slot], ph ^ 1, abort)) goto u_done;
                     tc_fence_after();        // order the stores after the MMAs that read this slot
                     tmem_st_32x32b_x32(a_addr, q0);

@@ -93,58 +93,189 @@ wq_status launch_pack(const void *W, int64_t n_groups, uint8_t *packed, float *s
 }
 
 // ------------------------------------------------------------------ small-M path
-template <int BITS, int NT>
-wq_status launch_smallm_nt(const wq::SmallMArgs &a, int splits, cudaStream_t st) {
-    constexpr int PF = wq::small_prefetch(BITS);
-    const size_t smem = wq::small_smem_bytes<NT>(PF);
-    static bool attr_done[kMaxDevices] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (!attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(wq::smallm_kernel<BITS, NT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smallm)");
-        e = cudaFuncSetAttribute(wq::smallm_kernel<BITS, NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        (void)e;
+constexpr uint32_t kSmemMax = 227 * 1024;        // dynamic shared memory per CTA on sm_100
+
+uint32_t align_u32(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
+// Stage and shared-memory layout of smallm_kernel for `rows` weight rows per stage and a
+// CTA range of `gcta` groups (`even`: every CTA of the launch has exactly gcta groups).
+// Chunk width gc: the largest candidate that keeps a ring of at least three stages (two at
+// one group per chunk); with an even split the candidates are the divisors of gcta, so no
+// chunk is short. gc * bits <= 64 keeps a weight box row within 256 32-bit words.
+template <int TOK>
+bool small_layout(int bits, int rows, int gcta, bool even, bool scale_tma, int sbox, wq::SmallMArgs &a,
+                  uint32_t *total) {
+    using T = wq::SmTok<TOK>;
+    const uint32_t tree = 4u * T::kNR * 32u * 4u;
+    const uint32_t part = align_u32((uint32_t)TOK * T::kPStride * 4u, 128);
+    const uint32_t bars = (2u * wq::kSmMaxStages + 4u) * 8u + 16u;
+    const uint32_t sres = scale_tma ? align_u32((uint32_t)rows * (uint32_t)sbox * 4u, 128) : 0u;
+    if (tree + part + bars + sres >= kSmemMax) return false;
+    const uint32_t budget = kSmemMax - tree - part - bars - sres;
+    for (int gc = std::min(gcta, 64 / bits); gc >= 1; --gc) {
+        if (even ? (gcta % gc != 0) : ((gc & (gc - 1)) != 0 || gc > 8)) continue;
+        const uint32_t w_bytes = align_u32((uint32_t)rows * (uint32_t)gc * 16u * (uint32_t)bits, 128);
+        const uint32_t x_bytes = align_u32((uint32_t)TOK * (uint32_t)gc * 256u, 128);
+        const uint32_t s_bytes = scale_tma ? 0u : align_u32((uint32_t)gc * (uint32_t)rows * 4u, 128);
+        const uint32_t stage = w_bytes + x_bytes + s_bytes;
+        const uint32_t stages = std::min<uint32_t>(wq::kSmMaxStages, budget / stage);
+        if (stages < 3 && !(gc == 1 && stages >= 2)) continue;
+        a.gc = gc;
+        a.stages = (int)stages;
+        a.srows = rows;
+        a.stage_bytes = stage;
+        a.off_x = w_bytes;
+        a.off_s = w_bytes + x_bytes;
+        a.scale_tma = scale_tma ? 1 : 0;
+        a.sbox = sbox;
+        a.off_sres = stages * stage;
+        a.off_tree = a.off_sres + sres;
+        a.off_part = a.off_tree + tree;
+        a.off_bar = a.off_part + part;
+        *total = a.off_bar + bars;
+        return true;
+    }
+    return false;
+}
+
+// Clusters of S CTAs that fit at once (one CTA per SM, the most shared memory), cached.
+template <int BITS, int TOK>
+int small_max_clusters(int dev, int S, int sm_count) {
+    static int cache[kMaxDevices][3] = {};
+    const int si = S == 1 ? 0 : (S == 2 ? 1 : 2);
+    if (cache[dev][si] != 0) return cache[dev][si];
+    int n = sm_count / S;
+    if (S > 1) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(S * (sm_count / S)));
+        cfg.blockDim = dim3(wq::kSmThreads);
+        cfg.dynamicSmemBytes = kSmemMax;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)S;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int q = 0;
+        if (cudaOccupancyMaxActiveClusters(&q, (void *)wq::smallm_kernel<BITS, TOK>, &cfg) != cudaSuccess) q = 0;
         cudaGetLastError();
+        n = std::min(n, q);
+    }
+    cache[dev][si] = n > 0 ? n : -1;
+    return cache[dev][si];
+}
+
+wq_status get_encoder();
+wq_status make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
+wq_status make_map_3d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, const uint64_t (&dims)[3],
+                      const uint64_t (&strides)[2], const uint32_t (&box)[3]);
+
+template <int BITS, int TOK>
+wq_status launch_smallm_tok(wq::SmallMArgs a, const uint8_t *packed, int dev, int sm_count, cudaStream_t st) {
+    using T = wq::SmTok<TOK>;
+    static bool attr_done[kMaxDevices] = {};
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(wq::smallm_kernel<BITS, TOK>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smallm)");
         attr_done[dev] = true;
     }
+    const int64_t U = (a.N + 15) / 16;
+    const int G = (int)(a.K / 128);
+    // cluster size S (K split) and cluster count C: the fewest items on the busiest CTA,
+    // items = (16-row units per cluster) x (groups per CTA); ties go to the smaller S
+    int bestS = 1, bestC = 1;
+    int64_t best = -1;
+    for (int S = 1; S <= 4; S *= 2) {
+        if (S > G) break;
+        const int mc = small_max_clusters<BITS, TOK>(dev, S, sm_count);
+        if (mc <= 0) continue;
+        const int C = (int)std::min<int64_t>(mc, U);
+        const int64_t cost = ((U + C - 1) / C) * ((G + S - 1) / S);
+        if (best < 0 || cost < best) { best = cost; bestS = S; bestC = C; }
+    }
+    a.S = bestS;
+    a.n_clusters = bestC;
+    const int rows = (int)std::min<int64_t>(T::kRP, (U + bestC - 1) / bestC) * 16;
+    const int gcta = (G + bestS - 1) / bestS;
+    const bool even = (G % bestS) == 0;
+    // resident steps by TMA: rows of G fp32 must be 16-byte multiples; the box covers the
+    // CTA's groups from the 4-aligned group below its first one
+    const int sbox = (gcta + 3 + 3) / 4 * 4;
+    bool scale_tma = (G % 4 == 0) && sbox <= 256 && (uint64_t)rows * sbox * 4 <= 48 * 1024;
+    uint32_t smem = 0;
+    if (!small_layout<TOK>(BITS, rows, gcta, even, scale_tma, sbox, a, &smem)) {
+        scale_tma = false;
+        if (!small_layout<TOK>(BITS, rows, gcta, even, false, sbox, a, &smem))
+            return fail(WQ_ERR_INVALID_ARG, "no shared-memory layout for the small-M kernel");
+    }
+    // TMA maps: packed as [N][K*b/32] 32-bit words (boxes of gc groups x 64/32/16 rows) and,
+    // for short chunks, as {16b bytes, G, N} one group at a time; x as {128 k, G, M};
+    // steps as [N][G] fp32
+    const uint64_t G64 = (uint64_t)G, kGB = 16u * BITS, row_bytes = (uint64_t)a.K * BITS / 8;
+    CUtensorMap pm64, pm32, pm16, pm_tail, xm_full, xm_tail, sm_map;
+    wq_status s;
+    const uint64_t pdims[3] = {kGB, G64, (uint64_t)a.N};
+    const uint64_t pstr[2] = {kGB, row_bytes};
+    const uint64_t xdims[3] = {128, G64, (uint64_t)a.M};
+    const uint64_t xstr[2] = {256, (uint64_t)a.K * 2};
+    const uint32_t pbox_t[3] = {(uint32_t)kGB, 1, 16};
+    const uint32_t xbox_f[3] = {128, (uint32_t)a.gc, (uint32_t)TOK}, xbox_t[3] = {128, 1, (uint32_t)TOK};
+    const uint32_t wbox = (uint32_t)a.gc * 4u * BITS;
+    if ((s = make_map_2d(&pm64, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, row_bytes / 4, (uint64_t)a.N, row_bytes, wbox, 64,
+                         CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK ||
+        (s = make_map_2d(&pm32, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, row_bytes / 4, (uint64_t)a.N, row_bytes, wbox, 32,
+                         CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK ||
+        (s = make_map_2d(&pm16, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, row_bytes / 4, (uint64_t)a.N, row_bytes, wbox, 16,
+                         CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK ||
+        (s = make_map_3d(&pm_tail, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, pdims, pstr, pbox_t)) != WQ_OK ||
+        (s = make_map_3d(&xm_full, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, xdims, xstr, xbox_f)) != WQ_OK ||
+        (s = make_map_3d(&xm_tail, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, xdims, xstr, xbox_t)) != WQ_OK)
+        return s;
+    if (scale_tma) {
+        if ((s = make_map_2d(&sm_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.scales, G64, (uint64_t)a.N, G64 * 4,
+                             (uint32_t)sbox, 16, CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK)
+            return s;
+    } else {
+        sm_map = pm16;   // not read by the kernel
+    }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((a.N + wq::kSmallRows - 1) / wq::kSmallRows), (unsigned)splits,
-                       (unsigned)((a.M + 8 * NT - 1) / (8 * NT)));
-    cfg.blockDim = dim3(wq::kSmallThreads);
+    cfg.gridDim = dim3((unsigned)(bestC * bestS));
+    cfg.blockDim = dim3(wq::kSmThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = (unsigned)splits;
+    attr[0].val.clusterDim.x = (unsigned)bestS;
+    attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, wq::smallm_kernel<BITS, NT>, a);
+    cfg.numAttrs = bestS > 1 ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, wq::smallm_kernel<BITS, TOK>, pm64, pm32, pm16, pm_tail, xm_full, xm_tail,
+                                       sm_map, a);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(smallm_kernel)");
     return check_launch("smallm_kernel");
 }
 
+// Up to 16 tokens per launch; more tokens take several launches.
 template <int BITS>
-wq_status launch_smallm(const wq::SmallMArgs &a, int splits, cudaStream_t st) {
-    if (a.M <= 8) return launch_smallm_nt<BITS, 1>(a, splits, st);
-    if (a.M <= 16) return launch_smallm_nt<BITS, 2>(a, splits, st);
-    return launch_smallm_nt<BITS, 4>(a, splits, st);
+wq_status launch_smallm(const wq::SmallMArgs &base, const uint8_t *packed, int dev, int sm_count, cudaStream_t st) {
+    for (int64_t m0 = 0; m0 < base.M; m0 += wq::kSmMaxTok) {
+        wq::SmallMArgs a = base;
+        a.M = std::min<int64_t>(wq::kSmMaxTok, base.M - m0);
+        a.x = base.x + m0 * base.K;
+        a.y = base.y + m0 * base.N;
+        if (base.t) a.t = base.t + m0 * wq::kTStrideSm;
+        wq_status s;
+        if (a.M <= 8) s = launch_smallm_tok<BITS, 8>(a, packed, dev, sm_count, st);
+        else s = launch_smallm_tok<BITS, 16>(a, packed, dev, sm_count, st);
+        if (s != WQ_OK) return s;
+    }
+    return WQ_OK;
 }
 
-int smallm_splits(int64_t M, int64_t N, int64_t K, int sm_count) {
-    const int64_t G = K / 128;
-    const int64_t slabs = (N + wq::kSmallRows - 1) / wq::kSmallRows;
-    const int64_t passes = (M + 31) / 32;
-    int s = 1;
-    // split K until about 4 CTAs per SM, at most 8 (portable cluster size), never past G
-    while (s < 8 && s < G && slabs * passes * s < 4 * (int64_t)sm_count) s *= 2;
-    return (int)std::min<int64_t>(s, G);
-}
-
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // ------------------------------------------------------------------ tensor-core path
 constexpr int64_t kSmallMThreshold = 32;
@@ -185,6 +316,8 @@ wq_status get_encoder() {
 
 wq_status make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    wq_status s = get_encoder();
+    if (s != WQ_OK) return s;
     const cuuint64_t dims[2] = {inner, outer};
     const cuuint64_t strides[1] = {row_bytes};
     const cuuint32_t box[2] = {box_inner, box_outer};
@@ -193,6 +326,21 @@ wq_status make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base
                           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(WQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return WQ_OK;
+}
+
+wq_status make_map_3d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, const uint64_t (&dims)[3],
+                      const uint64_t (&strides)[2], const uint32_t (&box)[3]) {
+    wq_status s = get_encoder();
+    if (s != WQ_OK) return s;
+    const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+    const cuuint64_t st[2] = {strides[0], strides[1]};
+    const cuuint32_t b[3] = {box[0], box[1], box[2]};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, dt, 3, const_cast<void *>(base), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(WQ_ERR_CUDA, "cuTensorMapEncodeTiled (3d) failed (%d)", (int)r);
     return WQ_OK;
 }
 
@@ -283,7 +431,7 @@ wq_status tc_linear(const TcArgs &a, int sm_count, cudaStream_t st) {
     }
 }
 
-size_t smallm_workspace(int64_t M, int rank) { return rank > 0 ? align_up((size_t)M * rank * 4, 256) : 0; }
+size_t smallm_workspace(int64_t M, int rank) { return tc_workspace_bytes(M, 0, 0, rank); }
 
 // ------------------------------------------------------------------ static scratch
 // Scratch for wq_linear_no_workspace: a file-scope device array. In host code its name is
@@ -411,27 +559,32 @@ wq_status wq_linear_ex(const void *x, int64_t M, int64_t K, const uint8_t *packe
 
     wq::SmallMArgs a{};
     a.x = static_cast<const uint16_t *>(x);
-    a.packed = packed;
     a.scales = scales;
     a.bias = static_cast<const uint16_t *>(bias);
     a.L2 = static_cast<const uint16_t *>(L2);
     a.y = static_cast<uint16_t *>(y);
     a.M = M; a.N = N; a.K = K; a.rank = rank;
+    if (M > (int64_t)INT32_MAX || N > (int64_t)INT32_MAX || K > (int64_t)INT32_MAX)
+        return fail(WQ_ERR_INVALID_ARG, "dimension above 2^31 on the small-M path");
     if (rank > 0) {
-        float *t = static_cast<float *>(workspace);
-        dim3 grid((unsigned)M, (unsigned)((rank + 31) / 32));
-        wq::lowrank_small_kernel<<<grid, 256, 0, st>>>(static_cast<const uint16_t *>(x),
-                                                        static_cast<const uint16_t *>(L1), t, K, rank);
-        if ((s = check_launch("lowrank_small_kernel")) != WQ_OK) return s;
+        // t = x L1 as [t_hi | t_lo] bf16 pairs, the same prepass as the tensor-core path
+        TcArgs ta{x, M, K, packed, scales, bits, N, L1, L2, rank, bias, y, workspace};
+        uint16_t *t = static_cast<uint16_t *>(workspace);
+        switch (rank) {
+            case 16: s = launch_prepass<16>(ta, t, info->sm_count, st); break;
+            case 32: s = launch_prepass<32>(ta, t, info->sm_count, st); break;
+            case 48: s = launch_prepass<48>(ta, t, info->sm_count, st); break;
+            default: s = launch_prepass<64>(ta, t, info->sm_count, st); break;
+        }
+        if (s != WQ_OK) return s;
         a.t = t;
     }
-    const int splits = smallm_splits(M, N, K, info->sm_count);
     switch (bits) {
-        case 3: return launch_smallm<3>(a, splits, st);
-        case 4: return launch_smallm<4>(a, splits, st);
-        case 5: return launch_smallm<5>(a, splits, st);
-        case 6: return launch_smallm<6>(a, splits, st);
-        default: return launch_smallm<7>(a, splits, st);
+        case 3: return launch_smallm<3>(a, packed, dev, info->sm_count, st);
+        case 4: return launch_smallm<4>(a, packed, dev, info->sm_count, st);
+        case 5: return launch_smallm<5>(a, packed, dev, info->sm_count, st);
+        case 6: return launch_smallm<6>(a, packed, dev, info->sm_count, st);
+        default: return launch_smallm<7>(a, packed, dev, info->sm_count, st);
     }
 }
 
