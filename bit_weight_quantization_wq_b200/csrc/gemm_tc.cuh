@@ -61,7 +61,7 @@ constexpr uint32_t kTcTmemCols = 512;
 constexpr uint32_t kTmemT0 = 0, kTmemA = 256;
 constexpr int kTStride = 128;             // row stride (elements) of the low-rank [t_hi | t_lo] buffer
 
-template <int BITS> struct TcStagesP { static constexpr int value = BITS <= 4 ? 8 : 6; };
+template <int BITS> struct TcStagesP { static constexpr int value = BITS <= 4 ? 8 : 5; };
 
 template <int BITS>
 struct TcLayout {
@@ -70,8 +70,10 @@ struct TcLayout {
     static constexpr uint32_t kPBytes = kTcBW * 16 * BITS;          // 128 rows x one group
     static constexpr uint32_t kOffX = 0;
     static constexpr uint32_t kOffP = kOffX + kTcStagesX * kXBytes;
-    static constexpr uint32_t kOffBar = kOffP + kSP * kPBytes;
-    static constexpr uint32_t kNumBars = 2 * kTcSlots + 2 * kSP + 2 + 2;
+    static constexpr uint32_t kOffL = kOffP + kSP * kPBytes;       // low-rank L2 tile [rank][128] bf16
+    static constexpr uint32_t kLBytes = 64 * kTcBW * 2;
+    static constexpr uint32_t kOffBar = kOffL + kLBytes;
+    static constexpr uint32_t kNumBars = 2 * kTcSlots + 2 * kSP + 2 + 2 + 2;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kBytes = kOffMisc + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;               // slack to align the base to 1024 B
@@ -85,6 +87,7 @@ struct TcParams {
     int64_t M, N, K;
     int rank;
     int tiles_m, tiles_n;
+    int l_tma;                // 1: the low-rank L2 tile of each weight tile arrives by TMA (l_map)
 };
 
 // k stages (64 wide) of the low-rank unit: [t_hi | t_lo] has 2 * rank columns.
@@ -93,7 +96,8 @@ __host__ __device__ constexpr int lowrank_stages(int rank) { return (2 * rank + 
 template <int BITS>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap p_map,
-                 const __grid_constant__ CUtensorMap t_map, const TcParams p) {
+                 const __grid_constant__ CUtensorMap t_map, const __grid_constant__ CUtensorMap l_map,
+                 const TcParams p) {
     using L = TcLayout<BITS>;
     constexpr int SP = L::kSP;
     constexpr int NWG = 4 * BITS + 1;
@@ -104,6 +108,8 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
     uint64_t *ready = bars, *consumed = ready + kTcSlots;
     uint64_t *p_full = consumed + kTcSlots, *p_empty = p_full + SP;
     uint64_t *t_full = p_empty + SP, *drain = t_full + 2;      // drain[2]: one per MMA thread
+    uint64_t *l_full = drain + 2, *l_empty = l_full + 1;        // low-rank L2 tile handoff
+    const uint16_t *l_tile = reinterpret_cast<const uint16_t *>(smem + L::kOffL);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
 
@@ -115,6 +121,8 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         for (int i = 0; i < 2; ++i) mbar_init(&t_full[i], 1);
         mbar_init(&drain[0], 1);
         mbar_init(&drain[1], 1);
+        mbar_init(l_full, 1);
+        mbar_init(l_empty, 4 * 32);
         *abort = 0;
         fence_barrier_init();
     }
@@ -165,7 +173,9 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         tma_prefetch_desc(&p_map);
         int armed[SP];
         for (int i = 0; i < SP; ++i) armed[i] = -1;
-        uint32_t s = 0, ph = 0;
+        if (p.l_tma) tma_prefetch_desc(&l_map);
+        uint32_t s = 0, ph = 0, lph = 0;
+        int l_armed = -1;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int nt = tile / p.tiles_m;
             for (int g = 0; g < G; ++g) {
@@ -175,11 +185,24 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                 tma_load_2d(smem + L::kOffP + s * L::kPBytes, &p_map, &p_full[s], g * 16 * BITS, nt * kTcBW);
                 if (++s == SP) { s = 0; ph ^= 1; }
             }
+            if (p.l_tma) {
+                // this tile's L2 columns, [rank][128 rows]; the tile's low-rank unit comes after all
+                // its groups, so the copy issued here lands long before it is read
+                if (!mbar_wait(l_empty, lph ^ 1, abort)) goto p_done;
+                mbar_arrive_expect_tx(l_full, (uint32_t)p.rank * kTcBW * 2);
+                l_armed = (int)lph;
+                tma_load_2d(smem + L::kOffL, &l_map, l_full, nt * kTcBW, 0);
+                lph ^= 1;
+            }
         }
     p_done:
         for (int i = 0; i < SP; ++i) {
             int local = 0;
             if (armed[i] >= 0) (void)mbar_wait(&p_full[i], (uint32_t)armed[i], &local);
+        }
+        if (l_armed >= 0) {
+            int local = 0;
+            (void)mbar_wait(l_full, (uint32_t)l_armed, &local);
         }
     } else if ((warp == 1 || warp == 3) && lane == 0) {
         // ---------------------------------------------------------- MMA issuers
@@ -223,7 +246,7 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         const int quarter = warp & 3;
         const int row_local = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        uint32_t sp = 0, pp = 0, unit = 0;
+        uint32_t sp = 0, pp = 0, unit = 0, lph = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int nt = tile / p.tiles_m;
             const int64_t n = (int64_t)nt * kTcBW + row_local;
@@ -261,7 +284,9 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                     tmem_st_32x32b_x32(a_addr + kTcBK / 2, q1);
                 } else {
                     // low-rank unit: A[n][k] = L2[k mod rank][n] for k < 2 rank (both halves of
-                    // [t_hi | t_lo] meet the same L2), zero beyond
+                    // [t_hi | t_lo] meet the same L2), zero beyond; from the shared-memory tile
+                    // when it came by TMA, else straight from global memory
+                    if (p.l_tma && !warp_wait(l_full, lph, abort)) goto u_done;
                     if (!warp_wait(&consumed[slot], ph ^ 1, abort)) goto u_done;
                     tc_fence_after();
                     const int nst = lowrank_stages(p.rank);
@@ -271,15 +296,25 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                         for (int i = 0; i < 32; ++i) {
                             const int k = st * kTcBK + 2 * i;
                             uint32_t v = 0;
-                            if (row_ok && k < 2 * p.rank) {
-                                const int j = k % p.rank;
-                                const uint32_t a = __ldg(p.L2 + (int64_t)j * p.N + n);
-                                const uint32_t b = __ldg(p.L2 + (int64_t)(j + 1) * p.N + n);
-                                v = a | (b << 16);
+                            if (k < 2 * p.rank) {
+                                const int j = k < p.rank ? k : k - p.rank;
+                                if (p.l_tma) {
+                                    v = (uint32_t)l_tile[j * kTcBW + row_local] | ((uint32_t)l_tile[(j + 1) * kTcBW + row_local] << 16);
+                                } else if (row_ok) {
+                                    v = (uint32_t)__ldg(p.L2 + (int64_t)j * p.N + n) |
+                                        ((uint32_t)__ldg(p.L2 + (int64_t)(j + 1) * p.N + n) << 16);
+                                }
                             }
                             q[i] = v;
                         }
                         tmem_st_32x32b_x32(a_addr + st * (kTcBK / 2), q);
+                    }
+                    if (p.l_tma) {
+                        // the tile is read: release it to the next tile's copy (per lane, after the
+                        // proxy fence, as for the packed stages)
+                        fence_proxy_async_smem();
+                        mbar_arrive(l_empty);
+                        lph ^= 1;
                     }
                 }
                 tmem_wait_st();

@@ -346,7 +346,7 @@ wq_status make_map_3d(CUtensorMap *map, CUtensorMapDataType dt, const void *base
 
 template <int BITS>
 wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &pm, const CUtensorMap &tm,
-                    int sm_count, cudaStream_t st) {
+                    const CUtensorMap &lm, int l_tma, int sm_count, cudaStream_t st) {
     using L = wq::TcLayout<BITS>;
     static bool attr_done[kMaxDevices] = {};
     int dev = 0;
@@ -365,9 +365,10 @@ wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &p
     p.M = a.M; p.N = a.N; p.K = a.K; p.rank = a.rank;
     p.tiles_m = (int)((a.M + wq::kTcBT - 1) / wq::kTcBT);
     p.tiles_n = (int)((a.N + wq::kTcBW - 1) / wq::kTcBW);
+    p.l_tma = l_tma;
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = std::min(tiles, sm_count);
-    wq::tc_linear_kernel<BITS><<<grid, wq::kTcThreads, L::kAlloc, st>>>(xm, pm, tm, p);
+    wq::tc_linear_kernel<BITS><<<grid, wq::kTcThreads, L::kAlloc, st>>>(xm, pm, tm, lm, p);
     return check_launch("tc_linear_kernel");
 }
 
@@ -375,8 +376,21 @@ template <int R>
 wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_t st) {
     const int64_t mtiles = (a.M + 63) / 64;
     const int64_t nkb = a.K / 64;
+    // The prepass is latency-bound (each CTA walks its K share one 64-k block at a time), so
+    // K is split (clusters of up to 16 CTAs, a non-portable size) until about eight CTAs per
+    // SM are in flight.
+    static bool attr_done[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(wq::lowrank_prepass_kernel<R>,
+                                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(lowrank_prepass_kernel)");
+        attr_done[dev] = true;
+    }
+    const int kmax = 16;
     int ks = 1;
-    while (ks < 8 && ks * 2 <= nkb && mtiles * ks < 2 * (int64_t)sm_count) ks *= 2;
+    while (ks < kmax && ks * 2 <= nkb && mtiles * ks < 8 * (int64_t)sm_count) ks *= 2;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)mtiles, (unsigned)ks, 1);
     cfg.blockDim = dim3(128);
@@ -400,7 +414,8 @@ wq_status tc_linear(const TcArgs &a, int sm_count, cudaStream_t st) {
     if (s != WQ_OK) return s;
     if (a.M > (int64_t)INT32_MAX || a.N > (int64_t)INT32_MAX || a.K > (int64_t)INT32_MAX)
         return fail(WQ_ERR_INVALID_ARG, "dimension above 2^31 on the tensor-core path");
-    CUtensorMap xm, pm, tm;
+    CUtensorMap xm, pm, tm, lm;
+    int l_tma = 0;
     if ((s = make_map_2d(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)a.K, (uint64_t)a.M,
                          (uint64_t)a.K * 2, wq::kTcBK, wq::kTcBT, CU_TENSOR_MAP_SWIZZLE_128B)) != WQ_OK)
         return s;
@@ -421,13 +436,21 @@ wq_status tc_linear(const TcArgs &a, int sm_count, cudaStream_t st) {
         if ((s = make_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, t, (uint64_t)wq::kTStride, (uint64_t)a.M,
                              (uint64_t)wq::kTStride * 2, wq::kTcBK, wq::kTcBT, CU_TENSOR_MAP_SWIZZLE_128B)) != WQ_OK)
             return s;
+        // L2 (rank x N) by TMA when its rows are 16-byte multiples: a [rank][128] tile per weight tile
+        if (a.N % 8 == 0) {
+            if ((s = make_map_2d(&lm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.L2, (uint64_t)a.N, (uint64_t)a.rank,
+                                 (uint64_t)a.N * 2, wq::kTcBW, (uint32_t)a.rank, CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK)
+                return s;
+            l_tma = 1;
+        }
     }
+    if (!l_tma) lm = xm;   // not read by the kernel
     switch (a.bits) {
-        case 3: return launch_tc<3>(a, xm, pm, tm, sm_count, st);
-        case 4: return launch_tc<4>(a, xm, pm, tm, sm_count, st);
-        case 5: return launch_tc<5>(a, xm, pm, tm, sm_count, st);
-        case 6: return launch_tc<6>(a, xm, pm, tm, sm_count, st);
-        default: return launch_tc<7>(a, xm, pm, tm, sm_count, st);
+        case 3: return launch_tc<3>(a, xm, pm, tm, lm, l_tma, sm_count, st);
+        case 4: return launch_tc<4>(a, xm, pm, tm, lm, l_tma, sm_count, st);
+        case 5: return launch_tc<5>(a, xm, pm, tm, lm, l_tma, sm_count, st);
+        case 6: return launch_tc<6>(a, xm, pm, tm, lm, l_tma, sm_count, st);
+        default: return launch_tc<7>(a, xm, pm, tm, lm, l_tma, sm_count, st);
     }
 }
 
