@@ -174,6 +174,38 @@ def run_step(wq, lins, ws, events=None):
             events[i][2].record()
 
 
+# ----------------------------------------------------------------------------- measured traffic
+
+TRAFFIC_PROFILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                               "wq_linear_traffic_flux3_m4096_r32.md")
+KERNEL_SOURCES = ("gemm_tc.cuh", "unpack.cuh", "common.cuh", "wq_api.cu")
+
+
+def kernel_source_digest() -> str:
+    import hashlib
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "bit_weight_quantization_wq_b200", "csrc")
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic():
+    """DRAM bytes per wq_linear call (prepass + tensor-core kernel, mean over the 3 shapes) from
+    the committed ncu summary, or None when the kernel sources changed since it was taken."""
+    import re
+    try:
+        text = open(TRAFFIC_PROFILE).read()
+    except OSError:
+        return None
+    m_b = re.search(r"^traffic_bytes_per_call:\s*([0-9.eE+]+)", text, re.M)
+    m_h = re.search(r"^source_digest:\s*([0-9a-f]+)", text, re.M)
+    if not m_b or not m_h or m_h.group(1) != kernel_source_digest():
+        return None
+    return float(m_b.group(1))
+
+
 # ----------------------------------------------------------------------------- oracle legs
 
 def oracle_sample(lins_host, rows_per_linear: int, pack_rows: int):
@@ -200,8 +232,12 @@ def oracle_sample(lins_host, rows_per_linear: int, pack_rows: int):
 def cpu_baseline(lins_host, budget_s: float = 12.0):
     import oracle
     prow = min(lin["N"] for lin in lins_host)
-    f, p, t = oracle_sample(lins_host, 8, prow)          # calibration
-    rows = int(max(8, min(2048, 8 * budget_s / max(t, 1e-3))))
+    # calibration: the sample costs a fixed quantize+pack part plus a per-token-row part
+    _, _, t8 = oracle_sample(lins_host, 8, prow)
+    _, _, t40 = oracle_sample(lins_host, 40, prow)
+    per_row = max((t40 - t8) / 32, 1e-5)
+    fixed = max(t8 - 8 * per_row, 0.0)
+    rows = int(max(8, min(4096, (budget_s - fixed) / per_row)))
     f, p, t = oracle_sample(lins_host, rows, prow)
     return {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
             "sample": (f"C oracle (fp32 quantize+pack, fp64 linear with the rank-32 branch) on {prow} weight rows "
@@ -300,7 +336,7 @@ def main_arm(args):
     peaks, peak_src = load_peaks()
     lin_tflops = step_flops / (lin_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": lin_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": lin_tflops / peaks["bf16_tflops"], "traffic": None,
+                "frac": lin_tflops / peaks["bf16_tflops"], "traffic": measured_traffic(),
                 "kernel": "wq_linear (lowrank_prepass_kernel + tc_linear_kernel<4>), mean over the 3 shapes",
                 "peak_source": f"{peak_src} bf16 dense (burst)"}
 
