@@ -423,6 +423,7 @@ def case_arm(args):
 
     pack:N,K,bits            quantize+pack of an N x K weight
     linear:M,N,K,bits,rank   quantized linear (bias included), path from --path
+    model:BLOCKS             quantize+pack of BLOCKS DiT blocks (10 tensors each, mixed widths)
     Inputs are seeded torch draws on the GPU (weights ~N(0, 0.02^2), x ~N(0, 1)).
     """
     import torch
@@ -455,6 +456,27 @@ def case_arm(args):
         run = lambda: wq.wq_linear(x, packed, scales, bits, N, L1=L1, L2=L2, bias=b, y=y, workspace=ws, path=args.path)
         work = {"flops": gemm_flops(N, K, M, rank), "weight_bytes": weight_bytes(N, K, bits),
                 "bytes": 2 * M * K + 2 * M * N + weight_bytes(N, K, bits) + 2 * rank * (K + N) + 2 * N}
+    elif kind == "model":
+        # whole-model quantize+pack: `blocks` DiT blocks of 8 x 5120x5120, 13824x5120 and
+        # 5120x13824 tensors, widths drawn i.i.d. from the mixed-precision histogram; every
+        # tensor distinct and resident (34 GB at 49 blocks), so each read comes from HBM
+        from bit_weight_quantization_wq_b200 import synth
+        (blocks,) = vals
+        tensors = []
+        for blk in range(blocks):
+            widths = synth.mixed_bits(len(synth.BLOCK_SHAPES), config=5, block=blk)
+            for (N, K), bits in zip(synth.BLOCK_SHAPES, widths):
+                W = torch.randn(N, K, device=dev, generator=g, dtype=torch.bfloat16) * 0.015
+                tensors.append((W, bits, torch.empty((N, K * bits // 8), dtype=torch.uint8, device=dev),
+                                torch.empty((N, K // 128), dtype=torch.float32, device=dev)))
+
+        def run():
+            for W, bits, packed, scales in tensors:
+                wq.wq_quantize_pack(W, bits, packed=packed, scales=scales)
+        params = sum(W.numel() for W, _, _, _ in tensors)
+        packed_b = sum(p.numel() + 4 * sc.numel() for _, _, p, sc in tensors)
+        work = {"params": params, "bytes": 2 * params + packed_b, "bf16_gb": 2 * params / 1e9,
+                "packed_gb": packed_b / 1e9, "tensors": len(tensors)}
     else:
         raise SystemExit(f"unknown case kind {kind!r}")
     # Each timed call starts with a cold L2: a 256 MB buffer (larger than the 126 MB L2) is
@@ -495,6 +517,9 @@ def case_arm(args):
         out["gparams"] = work["params"] / us / 1e3
         out["gbs"] = work["bytes"] / us / 1e3
         out["frac_hbm"] = out["gbs"] / peaks["hbm_gbs"]
+        for k in ("bf16_gb", "packed_gb", "tensors"):
+            if k in work:
+                out[k] = work[k]
     out["peak_source"] = src
     print(json.dumps(out), flush=True)
     return 0
@@ -509,7 +534,8 @@ def parse(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--case", default=None, help="time one shape: pack:N,K,bits or linear:M,N,K,bits,rank")
+    ap.add_argument("--case", default=None,
+                    help="time one shape: pack:N,K,bits, linear:M,N,K,bits,rank or model:BLOCKS")
     ap.add_argument("--path", default="auto", choices=["auto", "small_m", "tensor"], help="kernel family for --case linear")
     return ap.parse_args(argv)
 

@@ -133,3 +133,23 @@ def test_binding_refuses_missing_library(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "libwq.so"))
     with pytest.raises(RuntimeError, match="libwq.so not found"):
         B.lib()
+
+
+def test_model_packed_size_accounting():
+    """The 49-block tensor set (8 x 5120x5120, 13824x5120, 5120x13824 per block) with the
+    mixed-precision widths: the library's packed-size answers add up to the bitstream size
+    (b/8 bytes per weight) plus one fp32 step per 128 weights, against 2 bytes per weight in
+    bf16."""
+    from bit_weight_quantization_wq_b200 import synth
+    total_bf16 = total_packed = 0
+    for block in range(49):
+        widths = synth.mixed_bits(len(synth.BLOCK_SHAPES), config=5, block=block)
+        for (N, K), bits in zip(synth.BLOCK_SHAPES, widths):
+            total_bf16 += 2 * N * K
+            packed = B.lib().wq_packed_bytes(N, K, bits, 128)
+            steps = B.lib().wq_scales_count(N, K, 128)
+            assert packed == N * K * bits // 8 and steps == N * K // 128
+            total_packed += packed + 4 * steps
+    assert total_bf16 == 49 * 2 * (8 * 5120 * 5120 + 2 * 13824 * 5120)
+    ratio = total_packed / total_bf16
+    assert 0.25 < ratio < 0.40      # ~5 bits per weight on average
