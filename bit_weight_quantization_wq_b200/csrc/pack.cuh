@@ -50,7 +50,7 @@
 
 namespace wq {
 
-constexpr int kPackThreads = 256;
+constexpr int kPackThreads = 128;       // with 6 CTAs per SM (<= 80 registers): 24 warps of loads in flight
 constexpr int kPackUnroll = 2;          // 8-group blocks per warp per loop iteration
 constexpr int kPackGroupsPerWarp = 8 * kPackUnroll;
 
@@ -89,7 +89,7 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
 }
 
 template <int BITS>
-__global__ void __launch_bounds__(kPackThreads)
+__global__ void __launch_bounds__(kPackThreads, 6)
 quantize_pack_kernel(const uint16_t *__restrict__ W, int64_t n_groups,
                      uint8_t *__restrict__ packed, float *__restrict__ scales) {
     constexpr int kLevels = (1 << BITS) - 1;

@@ -86,7 +86,7 @@ wq_status launch_pack(const void *W, int64_t n_groups, uint8_t *packed, float *s
                       cudaStream_t st) {
     const int64_t per_block = (int64_t)wq::kPackGroupsPerWarp * (wq::kPackThreads / 32);
     const int64_t want = (n_groups + per_block - 1) / per_block;
-    const int grid = (int)std::min<int64_t>(want, (int64_t)sm_count * 8);
+    const int grid = (int)std::min<int64_t>(want, (int64_t)sm_count * 16);
     wq::quantize_pack_kernel<BITS><<<grid, wq::kPackThreads, 0, st>>>(
         static_cast<const uint16_t *>(W), n_groups, packed, scales);
     return check_launch("quantize_pack_kernel");
