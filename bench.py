@@ -222,7 +222,7 @@ def oracle_sample(lins_host, rows_per_linear: int, pack_rows: int):
         codes, scales = oracle.quantize(lin["R"][:n], BITS)
         oracle.pack(codes, BITS)
         deq = oracle.dequant(codes, scales, BITS)
-        rows = np.arange(rows_per_linear, dtype=np.int64) + 17 * i
+        rows = (np.arange(rows_per_linear, dtype=np.int64) + 17 * i) % lin["x"].shape[0]
         oracle.linear_rows(lin["x"], deq, lin["L1"], lin["L2"][:, :n], lin["bias"][:n], rows)
         flops += gemm_flops(n, K, rows_per_linear, RANK)
         params += n * K
