@@ -3,8 +3,8 @@
 
 One step = the whole hot path over the FLUX-like DiT linears (4-bit, group 128, rank-32
 bf16 branch, bias, M = 4096 tokens): for each of W 3072x3072, 12288x3072 and 3072x12288,
-quantize + pack the residual weight (wq_quantize_pack), then run the fused dequant-GEMM
-y = x deq(R)^T + (x L1) L2 + bias (wq_linear).
+quantize + pack the residual weights (one wq_quantize_pack_many call for the three), then
+run the fused dequant-GEMM y = x deq(R)^T + (x L1) L2 + bias (wq_linear) of each.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -161,17 +161,20 @@ def make_workload(device):
     return out
 
 
-def run_step(wq, lins, ws, events=None):
+def run_step(wq, lins, ws, pack, events=None):
+    """One step: quantize + pack the three residuals (one prepared wq_quantize_pack_many
+    call, a single launch), then the three quantized linears. events: [pack start, pack end,
+    end of linear 0, 1, 2]."""
+    if events is not None:
+        events[0].record()
+    pack()
+    if events is not None:
+        events[1].record()
     for i, d in enumerate(lins):
-        if events is not None:
-            events[i][0].record()
-        wq.wq_quantize_pack(d["R"], BITS, packed=d["packed"], scales=d["scales"])
-        if events is not None:
-            events[i][1].record()
         wq.wq_linear(d["x"], d["packed"], d["scales"], BITS, d["N"], L1=d["L1"], L2=d["L2"],
                      bias=d["bias"], y=d["y"], workspace=ws)
         if events is not None:
-            events[i][2].record()
+            events[2 + i].record()
 
 
 # ----------------------------------------------------------------------------- measured traffic
@@ -305,15 +308,16 @@ def main_arm(args):
     step_params = sum(d["N"] * d["K"] for d in lins)
     step_wbytes = sum(weight_bytes(d["N"], d["K"], BITS) for d in lins)
 
+    pack = wq.PackJobs([(d["R"], BITS, d["packed"], d["scales"]) for d in lins])
     for _ in range(args.warmup):
-        run_step(wq, lins, ws)
+        run_step(wq, lins, ws, pack)
     torch.cuda.synchronize()
     if wq.wq_device_status() != 0:
         raise RuntimeError("device status not clean after warm-up")
 
     # ---------------------------------------------------------------- timed region
     K = args.steps
-    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in lins] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 + len(lins))] for _ in range(K)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world, device)
     torch.cuda.synchronize()
@@ -321,15 +325,15 @@ def main_arm(args):
     with ClockSampler(device.index) as clocks:
         start.record()
         for k in range(K):
-            run_step(wq, lins, ws, ev[k])
+            run_step(wq, lins, ws, pack, ev[k])
         stop.record()
         torch.cuda.synchronize()
     launches = wq.wq_launch_count() - launches0
     barrier(world, device)
     step_ms = start.elapsed_time(stop) / K
     step_ms = max_over_ranks(step_ms, world, device)
-    pack_ms = sum(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(K) for i in range(len(lins))) / K
-    lin_ms = sum(ev[k][i][1].elapsed_time(ev[k][i][2]) for k in range(K) for i in range(len(lins))) / K
+    pack_ms = sum(ev[k][0].elapsed_time(ev[k][1]) for k in range(K)) / K
+    lin_ms = sum(ev[k][1].elapsed_time(ev[k][-1]) for k in range(K)) / K
     if wq.wq_device_status() != 0:
         raise RuntimeError("device status not clean after the timed region")
 
@@ -460,7 +464,9 @@ def case_arm(args):
 
     pack:N,K,bits            quantize+pack of an N x K weight
     linear:M,N,K,bits,rank   quantized linear (bias included), path from --path
-    model:BLOCKS             quantize+pack of BLOCKS DiT blocks (10 tensors each, mixed widths)
+    model:BLOCKS             quantize+pack of BLOCKS DiT blocks (10 tensors each, mixed widths), one
+                             wq_quantize_pack_many call
+    model_per_tensor:BLOCKS  the same tensors, one wq_quantize_pack call each
     Inputs are seeded torch draws on the GPU (weights ~N(0, 0.02^2), x ~N(0, 1)).
     """
     import torch
@@ -493,7 +499,7 @@ def case_arm(args):
         run = lambda: wq.wq_linear(x, packed, scales, bits, N, L1=L1, L2=L2, bias=b, y=y, workspace=ws, path=args.path)
         work = {"flops": gemm_flops(N, K, M, rank), "weight_bytes": weight_bytes(N, K, bits),
                 "bytes": 2 * M * K + 2 * M * N + weight_bytes(N, K, bits) + 2 * rank * (K + N) + 2 * N}
-    elif kind == "model":
+    elif kind in ("model", "model_per_tensor"):
         # whole-model quantize+pack: `blocks` DiT blocks of 8 x 5120x5120, 13824x5120 and
         # 5120x13824 tensors, widths drawn i.i.d. from the mixed-precision histogram; every
         # tensor distinct and resident (34 GB at 49 blocks), so each read comes from HBM
@@ -507,9 +513,12 @@ def case_arm(args):
                 tensors.append((W, bits, torch.empty((N, K * bits // 8), dtype=torch.uint8, device=dev),
                                 torch.empty((N, K // 128), dtype=torch.float32, device=dev)))
 
-        def run():
-            for W, bits, packed, scales in tensors:
-                wq.wq_quantize_pack(W, bits, packed=packed, scales=scales)
+        if kind == "model":
+            run = wq.PackJobs(tensors)              # one prepared call: a few launches per width
+        else:
+            def run():                              # one wq_quantize_pack call per tensor
+                for W, bits, packed, scales in tensors:
+                    wq.wq_quantize_pack(W, bits, packed=packed, scales=scales)
         params = sum(W.numel() for W, _, _, _ in tensors)
         packed_b = sum(p.numel() + 4 * sc.numel() for _, _, p, sc in tensors)
         work = {"params": params, "bytes": 2 * params + packed_b, "bf16_gb": 2 * params / 1e9,
@@ -572,7 +581,7 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--case", default=None,
-                    help="time one shape: pack:N,K,bits, linear:M,N,K,bits,rank or model:BLOCKS")
+                    help="time one shape: pack:N,K,bits, linear:M,N,K,bits,rank, model:BLOCKS or model_per_tensor:BLOCKS")
     ap.add_argument("--path", default="auto", choices=["auto", "small_m", "tensor"], help="kernel family for --case linear")
     return ap.parse_args(argv)
 

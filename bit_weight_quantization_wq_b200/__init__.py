@@ -8,6 +8,7 @@ library; the first ``wq_*`` call does, and raises if it is missing.
 from ._binding import (  # noqa: F401
     PATHS,
     SYMBOLS,
+    PackJobs,
     WQError,
     lib,
     status_string,
@@ -17,6 +18,7 @@ from ._binding import (  # noqa: F401
     wq_linear_workspace_bytes,
     wq_packed_bytes,
     wq_quantize_pack,
+    wq_quantize_pack_many,
     wq_scales_count,
     wq_selftest_bounded_wait,
     wq_version,

@@ -30,7 +30,7 @@ SYMBOLS = (
     "wq_version", "wq_packed_bytes", "wq_scales_count", "wq_quantize_pack",
     "wq_linear_workspace_bytes", "wq_linear", "wq_linear_ex", "wq_device_status",
     "wq_selftest_bounded_wait", "wq_status_string", "wq_last_error", "wq_launch_count",
-    "wq_linear_no_workspace",
+    "wq_linear_no_workspace", "wq_quantize_pack_many",
 )
 
 
@@ -41,6 +41,12 @@ class WQError(RuntimeError):
         if detail:
             msg += f": {detail}"
         super().__init__(msg)
+
+
+class PackJob(ctypes.Structure):
+    """wq_pack_job of include/wq.h."""
+    _fields_ = [("W", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("bits", ctypes.c_int),
+                ("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
 
 
 _lib = None
@@ -75,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.wq_launch_count.argtypes, L.wq_launch_count.restype = [], ctypes.c_uint64
         L.wq_linear_no_workspace.argtypes = [p, i64, i64, p, p, i32, i32, i64, p, p, i32, p, p, p]
         L.wq_linear_no_workspace.restype = i32
+        L.wq_quantize_pack_many.argtypes = [ctypes.POINTER(PackJob), i32, i32, p]
+        L.wq_quantize_pack_many.restype = i32
         _lib = L
     return _lib
 
@@ -198,3 +206,52 @@ def wq_launch_count() -> int:
 
 def wq_selftest_bounded_wait(timeout_us: int, stream=None) -> int:
     return int(lib().wq_selftest_bounded_wait(timeout_us, _stream(stream)))
+
+
+class PackJobs:
+    """A prepared wq_quantize_pack_many call over many weights, each at its own width.
+
+    ``jobs``: iterable of ``(W, bits)`` or ``(W, bits, packed, scales)``, W an (N, K) bf16
+    CUDA tensor; missing outputs are allocated here. The descriptors are marshalled once, so
+    calling the object again (e.g. inside a timed loop) only crosses the C ABI. The tensors
+    are referenced for the object's lifetime. ``outputs``: one ``(packed, scales)`` per job.
+    """
+
+    def __init__(self, jobs, group: int = 128):
+        import torch
+        self.group = group
+        self.outputs = []
+        self._inputs = []
+        descs = []
+        for i, job in enumerate(list(jobs)):
+            if len(job) == 2:
+                (W, bits), packed, scales = job, None, None
+            else:
+                W, bits, packed, scales = job
+            _dev(W, f"jobs[{i}].W", torch.bfloat16)
+            if W.dim() != 2:
+                raise ValueError(f"jobs[{i}].W must be 2-D (N, K)")
+            N, K = W.shape
+            bits = int(bits)
+            if packed is None:
+                packed = torch.empty((N, K * bits // 8), dtype=torch.uint8, device=W.device)
+            if scales is None:
+                scales = torch.empty((N, max(K // group, 0)), dtype=torch.float32, device=W.device)
+            _dev(packed, f"jobs[{i}].packed", torch.uint8, (N, K * bits // 8))
+            _dev(scales, f"jobs[{i}].scales", torch.float32, (N, max(K // group, 0)))
+            self._inputs.append(W)
+            self.outputs.append((packed, scales))
+            descs.append(PackJob(W.data_ptr(), N, K, bits, packed.data_ptr(), scales.data_ptr()))
+        self._n = len(descs)
+        self._arr = (PackJob * max(1, self._n))(*descs)
+
+    def __call__(self, stream=None):
+        st = lib().wq_quantize_pack_many(self._arr, self._n, self.group, _stream(stream))
+        _check(st, "wq_quantize_pack_many")
+        return self.outputs
+
+
+def wq_quantize_pack_many(jobs, group: int = 128, stream=None):
+    """Quantize + pack many (N, K) bf16 weights, each at its own width, in a few launches.
+    ``jobs`` as for :class:`PackJobs`. Returns one ``(packed, scales)`` per job."""
+    return PackJobs(jobs, group)(stream)

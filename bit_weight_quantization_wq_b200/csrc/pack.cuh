@@ -8,7 +8,9 @@
 // Layout: the W rows are contiguous 128-element groups, so group G = n * (K/128) + g sits
 // at bf16 offset 128 G, its packed bytes at 16*b*G and its scale at G. The kernel is a flat
 // grid-stride loop over groups: four lanes own one group, each lane 32 consecutive weights
-// (64 bytes) and therefore exactly 4*b output bytes (b whole words).
+// (64 bytes) and therefore exactly 4*b output bytes (b whole words). A warp takes 16 groups
+// at a time (pack_block); quantize_pack_many_kernel runs the same blocks over the groups of
+// up to 64 tensors of one width, one launch for all of them.
 //
 // The kernel is HBM-bound only if it stays under ~8 instructions per weight, so every step
 // is chosen for its instruction count:
@@ -89,9 +91,16 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
 }
 
 template <int BITS>
-__global__ void __launch_bounds__(kPackThreads, 6)
-quantize_pack_kernel(const uint16_t *__restrict__ W, int64_t n_groups,
-                     uint8_t *__restrict__ packed, float *__restrict__ scales) {
+__host__ __device__ constexpr int pack_stage_words() { return BITS == 4 ? 1 : kPackGroupsPerWarp * 4 * BITS; }
+
+// One warp quantizes and packs the kPackGroupsPerWarp groups [g0, g0 + 16) of one tensor
+// (groups at or past n_groups are skipped). stage_w: the warp's pack_stage_words<BITS>()
+// words of shared memory (16-byte aligned), used to turn the lanes' b-word slices into
+// 16-byte stores.
+template <int BITS>
+__device__ __forceinline__ void pack_block(const uint16_t *__restrict__ W, int64_t n_groups,
+                                           uint8_t *__restrict__ packed, float *__restrict__ scales,
+                                           int64_t g0, uint32_t *stage_w, int lane) {
     constexpr int kLevels = (1 << BITS) - 1;
     constexpr int kOff = 1 << (BITS - 1);
     constexpr int kGroupBytes = 16 * BITS;
@@ -103,117 +112,159 @@ quantize_pack_kernel(const uint16_t *__restrict__ W, int64_t n_groups,
     constexpr float kMagicB = 8388608.0f + (float)(kOff * ((1 << BITS) + 1));
     constexpr float kPow = (float)(1 << BITS);
     constexpr uint32_t kMask2 = (1u << (2 * BITS)) - 1u;
-    constexpr int kStageWords = (BITS == 4) ? 1 : GW * 4 * BITS;
-    __shared__ __align__(16) uint32_t stage[kPackThreads / 32][kStageWords];
-
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gi = lane >> 2, l4 = lane & 3;
-    const int64_t warp_id = (int64_t)blockIdx.x * (kPackThreads / 32) + warp;
-    const int64_t n_warps = (int64_t)gridDim.x * (kPackThreads / 32);
 
-    for (int64_t g0 = warp_id * GW; g0 < n_groups; g0 += n_warps * GW) {
-        uint32_t w[U][16];
+    uint32_t w[U][16];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t g = g0 + 8 * u + gi;
-            const uint16_t *src = W + g * 128 + l4 * 32;
+    for (int u = 0; u < U; ++u) {
+        const int64_t g = g0 + 8 * u + gi;
+        const uint16_t *src = W + g * 128 + l4 * 32;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 v = (g < n_groups) ? ldg_nc_v4(src + 8 * i) : make_uint4(0, 0, 0, 0);
-                w[u][4 * i] = v.x; w[u][4 * i + 1] = v.y; w[u][4 * i + 2] = v.z; w[u][4 * i + 3] = v.w;
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t g = g0 + 8 * u + gi;
-            // ---- abs_max of the group (bf16 magnitudes; the max tree keeps only |.|)
-            uint32_t m8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) m8[i] = bf16x2_maxabs(w[u][2 * i], w[u][2 * i + 1]);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) m8[i] = bf16x2_maxabs(m8[i], m8[i + 4]);
-            m8[0] = bf16x2_maxabs(m8[0], m8[2]);
-            m8[1] = bf16x2_maxabs(m8[1], m8[3]);
-            const uint32_t m2 = bf16x2_maxabs(m8[0], m8[1]) & 0x7FFF7FFFu;
-            uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
-            m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-            const float abs_max = __uint_as_float(m << 16);
-            // ---- step = RN(2 s / L), s = RN(abs_max * 1.01)
-            const float two = __fmul_rn(2.0f, __fmul_rn(abs_max, 1.01f));
-            float step;
-            if (two >= 7.52316384526264e-37f && two <= 1.329227995784916e36f) {   // [2^-120, 2^120]
-                const float q0 = __fmul_rn(two, kInvL);
-                const float r = __fmaf_rn(-q0, kL, two);
-                step = __fmaf_rn(r, kInvL, q0);
-            } else {
-                step = __fdiv_rn(two, kL);
-            }
-            float inv = (step == 0.0f) ? 0.0f : __frcp_rn(step);
-            bool near = !(inv <= 3.402823466e38f);           // 1/step overflowed: divide always
-            if (near) inv = 0.0f;
-            // ---- quantize, two weights per instruction
-            const uint64_t inv2 = f2(inv, inv), magic = f2(kMagicA, kMagicB);
-            // pair fields: the low 2b bits of F[i] = code(2i) << b | code(2i+1)
-            uint32_t F[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint64_t x2 = (uint64_t)(w[u][i] << 16) | ((uint64_t)(w[u][i] & 0xFFFF0000u) << 32);
-                const uint64_t r2 = mul2(x2, inv2);
-                const uint64_t t2 = add2(r2, magic);
-                const uint64_t q2 = sub2(t2, magic);
-                const uint64_t e2 = sub2(r2, q2);
-                near |= (fabsf(f2_lo(e2)) > 0.49996f) | (fabsf(f2_hi(e2)) > 0.49996f);
-                F[i] = __float_as_uint(__fmaf_rn(f2_lo(q2), kPow, f2_hi(t2)));
-            }
-            if (near) {
-                // rare: a product close to a half-integer (or a huge 1/step): IEEE division
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float xa = __uint_as_float(w[u][i] << 16), xb = __uint_as_float(w[u][i] & 0xFFFF0000u);
-                    const float ra = (step == 0.0f) ? 0.0f : __fdiv_rn(xa, step);
-                    const float rb = (step == 0.0f) ? 0.0f : __fdiv_rn(xb, step);
-                    const float qa = __fsub_rn(__fadd_rn(ra, kMagicA), kMagicA);
-                    F[i] = __float_as_uint(__fmaf_rn(qa, kPow, __fadd_rn(rb, kMagicB)));
-                }
-            }
-            if (l4 == 0 && g < n_groups) scales[g] = step;
-            if constexpr (BITS == 4) {
-                // a pair field is one whole byte (bits 8..22 of the float are zero)
-                uint32_t o[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    o[k] = __byte_perm(__byte_perm(F[4 * k], F[4 * k + 1], 0x0040u),
-                                       __byte_perm(F[4 * k + 2], F[4 * k + 3], 0x0040u), 0x5410u);
-                if (g < n_groups)
-                    *reinterpret_cast<uint4 *>(packed + g * kGroupBytes + l4 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
-            } else {
-                // quad fields (4 codes, 4b bits), placed into the 32b-bit stream number whose
-                // most significant bits hold the first code; memory order is big-endian
-                uint32_t Nw[BITS];
-#pragma unroll
-                for (int k = 0; k < BITS; ++k) Nw[k] = 0;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t T = ((F[2 * j] & kMask2) << (2 * BITS)) | (F[2 * j + 1] & kMask2);
-                    const int o = 4 * BITS * (7 - j), wd = o / 32, sh = o % 32;
-                    Nw[wd] |= T << sh;
-                    if (sh + 4 * BITS > 32) Nw[wd + 1] |= T >> (32 - sh);
-                }
-                uint32_t *dst = stage[warp] + (8 * u + gi) * 4 * BITS + l4 * BITS;
-#pragma unroll
-                for (int k = 0; k < BITS; ++k) dst[k] = __byte_perm(Nw[BITS - 1 - k], 0, 0x0123u);
-            }
-        }
-        if constexpr (BITS != 4) {
-            __syncwarp();
-            const int64_t valid = min((int64_t)GW, n_groups - g0);
-            const int chunks = (int)(valid * kGroupBytes / 16);
-            uint4 *out = reinterpret_cast<uint4 *>(packed + g0 * kGroupBytes);
-            for (int c = lane; c < chunks; c += 32) out[c] = reinterpret_cast<const uint4 *>(stage[warp])[c];
-            __syncwarp();
+        for (int i = 0; i < 4; ++i) {
+            const uint4 v = (g < n_groups) ? ldg_nc_v4(src + 8 * i) : make_uint4(0, 0, 0, 0);
+            w[u][4 * i] = v.x; w[u][4 * i + 1] = v.y; w[u][4 * i + 2] = v.z; w[u][4 * i + 3] = v.w;
         }
     }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int64_t g = g0 + 8 * u + gi;
+        // ---- abs_max of the group (bf16 magnitudes; the max tree keeps only |.|)
+        uint32_t m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = bf16x2_maxabs(w[u][2 * i], w[u][2 * i + 1]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m8[i] = bf16x2_maxabs(m8[i], m8[i + 4]);
+        m8[0] = bf16x2_maxabs(m8[0], m8[2]);
+        m8[1] = bf16x2_maxabs(m8[1], m8[3]);
+        const uint32_t m2 = bf16x2_maxabs(m8[0], m8[1]) & 0x7FFF7FFFu;
+        uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        const float abs_max = __uint_as_float(m << 16);
+        // ---- step = RN(2 s / L), s = RN(abs_max * 1.01)
+        const float two = __fmul_rn(2.0f, __fmul_rn(abs_max, 1.01f));
+        float step;
+        if (two >= 7.52316384526264e-37f && two <= 1.329227995784916e36f) {   // [2^-120, 2^120]
+            const float q0 = __fmul_rn(two, kInvL);
+            const float r = __fmaf_rn(-q0, kL, two);
+            step = __fmaf_rn(r, kInvL, q0);
+        } else {
+            step = __fdiv_rn(two, kL);
+        }
+        float inv = (step == 0.0f) ? 0.0f : __frcp_rn(step);
+        bool near = !(inv <= 3.402823466e38f);           // 1/step overflowed: divide always
+        if (near) inv = 0.0f;
+        // ---- quantize, two weights per instruction
+        const uint64_t inv2 = f2(inv, inv), magic = f2(kMagicA, kMagicB);
+        // pair fields: the low 2b bits of F[i] = code(2i) << b | code(2i+1)
+        uint32_t F[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint64_t x2 = (uint64_t)(w[u][i] << 16) | ((uint64_t)(w[u][i] & 0xFFFF0000u) << 32);
+            const uint64_t r2 = mul2(x2, inv2);
+            const uint64_t t2 = add2(r2, magic);
+            const uint64_t q2 = sub2(t2, magic);
+            const uint64_t e2 = sub2(r2, q2);
+            near |= (fabsf(f2_lo(e2)) > 0.49996f) | (fabsf(f2_hi(e2)) > 0.49996f);
+            F[i] = __float_as_uint(__fmaf_rn(f2_lo(q2), kPow, f2_hi(t2)));
+        }
+        if (near) {
+            // rare: a product close to a half-integer (or a huge 1/step): IEEE division
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float xa = __uint_as_float(w[u][i] << 16), xb = __uint_as_float(w[u][i] & 0xFFFF0000u);
+                const float ra = (step == 0.0f) ? 0.0f : __fdiv_rn(xa, step);
+                const float rb = (step == 0.0f) ? 0.0f : __fdiv_rn(xb, step);
+                const float qa = __fsub_rn(__fadd_rn(ra, kMagicA), kMagicA);
+                F[i] = __float_as_uint(__fmaf_rn(qa, kPow, __fadd_rn(rb, kMagicB)));
+            }
+        }
+        if (l4 == 0 && g < n_groups) scales[g] = step;
+        if constexpr (BITS == 4) {
+            // a pair field is one whole byte (bits 8..22 of the float are zero)
+            uint32_t o[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                o[k] = __byte_perm(__byte_perm(F[4 * k], F[4 * k + 1], 0x0040u),
+                                   __byte_perm(F[4 * k + 2], F[4 * k + 3], 0x0040u), 0x5410u);
+            if (g < n_groups)
+                *reinterpret_cast<uint4 *>(packed + g * kGroupBytes + l4 * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+        } else {
+            // quad fields (4 codes, 4b bits), placed into the 32b-bit stream number whose
+            // most significant bits hold the first code; memory order is big-endian
+            uint32_t Nw[BITS];
+#pragma unroll
+            for (int k = 0; k < BITS; ++k) Nw[k] = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t T = ((F[2 * j] & kMask2) << (2 * BITS)) | (F[2 * j + 1] & kMask2);
+                const int o = 4 * BITS * (7 - j), wd = o / 32, sh = o % 32;
+                Nw[wd] |= T << sh;
+                if (sh + 4 * BITS > 32) Nw[wd + 1] |= T >> (32 - sh);
+            }
+            uint32_t *dst = stage_w + (8 * u + gi) * 4 * BITS + l4 * BITS;
+#pragma unroll
+            for (int k = 0; k < BITS; ++k) dst[k] = __byte_perm(Nw[BITS - 1 - k], 0, 0x0123u);
+        }
+    }
+    if constexpr (BITS != 4) {
+        __syncwarp();
+        const int64_t valid = min((int64_t)GW, n_groups - g0);
+        const int chunks = (int)(valid * kGroupBytes / 16);
+        uint4 *out = reinterpret_cast<uint4 *>(packed + g0 * kGroupBytes);
+        for (int c = lane; c < chunks; c += 32) out[c] = reinterpret_cast<const uint4 *>(stage_w)[c];
+        __syncwarp();
+    }
 }
+
+// One tensor: a flat grid-stride loop over its groups.
+template <int BITS>
+__global__ void __launch_bounds__(kPackThreads, 6)
+quantize_pack_kernel(const uint16_t *__restrict__ W, int64_t n_groups,
+                     uint8_t *__restrict__ packed, float *__restrict__ scales) {
+    __shared__ __align__(16) uint32_t stage[kPackThreads / 32][pack_stage_words<BITS>()];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t warp_id = (int64_t)blockIdx.x * (kPackThreads / 32) + warp;
+    const int64_t n_warps = (int64_t)gridDim.x * (kPackThreads / 32);
+    for (int64_t g0 = warp_id * kPackGroupsPerWarp; g0 < n_groups; g0 += n_warps * kPackGroupsPerWarp)
+        pack_block<BITS>(W, n_groups, packed, scales, g0, stage[warp], lane);
+}
+
+// Many tensors of one width in one launch (the mixed-precision article quantizes a whole
+// model tensor by tensor, each at its own width: one launch per tensor would pay a grid's
+// fill and drain per tensor). Segment i's groups occupy the virtual range
+// [vbegin[i], vbegin[i+1]), its group count rounded up to a multiple of kPackGroupsPerWarp,
+// so a warp's block of groups never straddles two tensors.
+constexpr int kPackMaxSegs = 64;
+struct PackSegments {
+    int n;                                   // segments in this launch, 1..kPackMaxSegs
+    int64_t vbegin[kPackMaxSegs + 1];        // vbegin[n] = end of the virtual range
+    int64_t n_groups[kPackMaxSegs];
+    const uint16_t *W[kPackMaxSegs];
+    uint8_t *packed[kPackMaxSegs];
+    float *scales[kPackMaxSegs];
+};
+
+template <int BITS>
+__global__ void __launch_bounds__(kPackThreads, 6)
+quantize_pack_many_kernel(const __grid_constant__ PackSegments segs) {
+    __shared__ __align__(16) uint32_t stage[kPackThreads / 32][pack_stage_words<BITS>()];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t warp_id = (int64_t)blockIdx.x * (kPackThreads / 32) + warp;
+    const int64_t n_warps = (int64_t)gridDim.x * (kPackThreads / 32);
+    const int64_t v_end = segs.vbegin[segs.n];
+    for (int64_t v0 = warp_id * kPackGroupsPerWarp; v0 < v_end; v0 += n_warps * kPackGroupsPerWarp) {
+        // the block's segment = the number of segments that end at or before v0
+        int s = 0;
+#pragma unroll
+        for (int base = 0; base < kPackMaxSegs; base += 32) {
+            const int j = base + lane;
+            s += __popc(__ballot_sync(0xffffffffu, j < segs.n && segs.vbegin[j + 1] <= v0));
+        }
+        pack_block<BITS>(segs.W[s], segs.n_groups[s], segs.packed[s], segs.scales[s], v0 - segs.vbegin[s],
+                         stage[warp], lane);
+    }
+}
+
 
 }  // namespace wq

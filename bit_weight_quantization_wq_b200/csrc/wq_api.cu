@@ -92,6 +92,38 @@ wq_status launch_pack(const void *W, int64_t n_groups, uint8_t *packed, float *s
     return check_launch("quantize_pack_kernel");
 }
 
+// The jobs of one width, packed by quantize_pack_many_kernel in launches of up to
+// kPackMaxSegs tensors (in the order given; empty jobs are skipped).
+template <int BITS>
+wq_status launch_pack_many(const wq_pack_job *jobs, int n_jobs, int sm_count, cudaStream_t st) {
+    constexpr int64_t GW = wq::kPackGroupsPerWarp;
+    const int64_t per_block = GW * (wq::kPackThreads / 32);
+    wq::PackSegments segs;
+    int i = 0;
+    while (i < n_jobs) {
+        segs.n = 0;
+        segs.vbegin[0] = 0;
+        for (; i < n_jobs && segs.n < wq::kPackMaxSegs; ++i) {
+            const wq_pack_job &j = jobs[i];
+            if (j.bits != BITS || j.N == 0 || j.K == 0) continue;
+            const int k = segs.n++;
+            const int64_t n_groups = j.N * (j.K / 128);
+            segs.n_groups[k] = n_groups;
+            segs.W[k] = static_cast<const uint16_t *>(j.W);
+            segs.packed[k] = j.packed;
+            segs.scales[k] = j.scales;
+            segs.vbegin[k + 1] = segs.vbegin[k] + (n_groups + GW - 1) / GW * GW;
+        }
+        if (segs.n == 0) break;
+        const int64_t want = (segs.vbegin[segs.n] + per_block - 1) / per_block;
+        const int grid = (int)std::min<int64_t>(want, (int64_t)sm_count * 16);
+        wq::quantize_pack_many_kernel<BITS><<<grid, wq::kPackThreads, 0, st>>>(segs);
+        const wq_status s = check_launch("quantize_pack_many_kernel");
+        if (s != WQ_OK) return s;
+    }
+    return WQ_OK;
+}
+
 // ------------------------------------------------------------------ small-M path
 constexpr uint32_t kSmemMax = 227 * 1024;        // dynamic shared memory per CTA on sm_100
 
@@ -536,6 +568,38 @@ wq_status wq_quantize_pack(const void *W, int64_t N, int64_t K, int bits, int gr
         case 6: return launch_pack<6>(W, n_groups, packed, scales, info->sm_count, st);
         default: return launch_pack<7>(W, n_groups, packed, scales, info->sm_count, st);
     }
+}
+
+wq_status wq_quantize_pack_many(const wq_pack_job *jobs, int n_jobs, int group, wq_stream_t stream) {
+    g_last_error[0] = 0;
+    if (group != 128) return fail(WQ_ERR_UNSUPPORTED_GROUP, "group=%d", group);
+    if (n_jobs < 0) return fail(WQ_ERR_INVALID_ARG, "n_jobs=%d", n_jobs);
+    if (n_jobs == 0) return WQ_OK;
+    if (!jobs) return fail(WQ_ERR_INVALID_ARG, "NULL job array");
+    bool any = false;
+    for (int i = 0; i < n_jobs; ++i) {
+        const wq_pack_job &j = jobs[i];
+        if (j.bits < 3 || j.bits > 7) return fail(WQ_ERR_UNSUPPORTED_BITS, "job %d: bits=%d", i, j.bits);
+        if (j.N < 0 || j.K < 0)
+            return fail(WQ_ERR_INVALID_ARG, "job %d: negative size N=%lld K=%lld", i, (long long)j.N, (long long)j.K);
+        if (j.K % 128 != 0) return fail(WQ_ERR_INVALID_ARG, "job %d: K=%lld is not a multiple of 128", i, (long long)j.K);
+        if (j.N == 0 || j.K == 0) continue;
+        if (!j.W || !j.packed || !j.scales) return fail(WQ_ERR_INVALID_ARG, "job %d: NULL tensor pointer", i);
+        if (!aligned16(j.W) || !aligned16(j.packed) || !aligned16(j.scales))
+            return fail(WQ_ERR_MISALIGNED, "job %d: W/packed/scales must be 16-byte aligned", i);
+        any = true;
+    }
+    if (!any) return WQ_OK;
+    int dev;
+    const DeviceInfo *info;
+    wq_status s = current_device(&dev, &info);
+    if (s != WQ_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if ((s = launch_pack_many<3>(jobs, n_jobs, info->sm_count, st)) != WQ_OK) return s;
+    if ((s = launch_pack_many<4>(jobs, n_jobs, info->sm_count, st)) != WQ_OK) return s;
+    if ((s = launch_pack_many<5>(jobs, n_jobs, info->sm_count, st)) != WQ_OK) return s;
+    if ((s = launch_pack_many<6>(jobs, n_jobs, info->sm_count, st)) != WQ_OK) return s;
+    return launch_pack_many<7>(jobs, n_jobs, info->sm_count, st);
 }
 
 size_t wq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int rank) {

@@ -94,6 +94,31 @@ WQ_API int64_t wq_scales_count(int64_t N, int64_t K, int group);
 WQ_API wq_status wq_quantize_pack(const void *W, int64_t N, int64_t K, int bits, int group,
                            uint8_t *packed, float *scales, wq_stream_t stream);
 
+/* One tensor of a wq_quantize_pack_many call: the arguments of one wq_quantize_pack. */
+typedef struct {
+    const void *W;        /* N x K bf16, device */
+    int64_t N, K;         /* K a multiple of 128; N == 0 or K == 0: nothing to do */
+    int bits;             /* 3..7, per tensor */
+    uint8_t *packed;      /* N x (K*bits/8) bytes, device */
+    float *scales;        /* N x (K/128) fp32, device */
+} wq_pack_job;
+
+/*
+ * Quantize and pack many tensors, each at its own width: the whole-model step of [PG]
+ * sec. 3.2 (every tensor gets its own bit width, 3..7) followed by sec. 3.1 and 3.3 for each.
+ *   jobs    in : host array of n_jobs descriptors (read during the call only; the library
+ *                keeps no pointer to it). n_jobs == 0 is a no-op.
+ *   group      : must be 128.
+ * Each job's outputs are bit-identical to those of wq_quantize_pack on the same arguments.
+ * The jobs' output buffers must not overlap one another or any job's W; the order in which
+ * the jobs run is unspecified. Tensors of one width are packed together, up to 64 per kernel
+ * launch, so a model's ~500 tensors take about a dozen launches instead of ~500.
+ * Every job is checked before anything is launched: the first bad job's status is returned
+ * (wq_last_error() names it) and nothing runs. A launch failure returns WQ_ERR_CUDA; the
+ * launches before it have been queued.
+ */
+WQ_API wq_status wq_quantize_pack_many(const wq_pack_job *jobs, int n_jobs, int group, wq_stream_t stream);
+
 /* Workspace bytes wq_linear / wq_linear_ex need for these sizes on any path
  * (0 if none; the caller then may pass NULL). */
 WQ_API size_t wq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int rank);

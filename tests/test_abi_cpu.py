@@ -29,7 +29,7 @@ def header_functions():
 
 def test_exports_match_header(L):
     declared = header_functions()
-    assert len(declared) == 13
+    assert len(declared) == 14
     out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
     exported = sorted(line.split()[-1] for line in out.splitlines() if line.split()[-1].startswith("wq_"))
@@ -84,6 +84,54 @@ def test_quantize_pack_argument_checks(L):
     assert _qp(L, 0, 0, 128, 4, 128, 0, 0) == B.WQ_OK
 
 
+def _jobs(*specs):
+    """specs: (W, N, K, bits, packed, scales) tuples of fake device addresses."""
+    arr = (B.PackJob * max(1, len(specs)))(*[B.PackJob(*sp) for sp in specs])
+    return arr, len(specs)
+
+
+def _many(L, arr, n, group=128):
+    return L.wq_quantize_pack_many(arr, n, group, None)
+
+
+def test_pack_job_struct_matches_header(tmp_path):
+    """The binding's PackJob has the size and field offsets of the C wq_pack_job."""
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "wq.h"\n'
+        'int main(void) { printf("%zu %zu %zu %zu %zu %zu %zu\\n", sizeof(wq_pack_job),'
+        ' offsetof(wq_pack_job, W), offsetof(wq_pack_job, N), offsetof(wq_pack_job, K),'
+        ' offsetof(wq_pack_job, bits), offsetof(wq_pack_job, packed), offsetof(wq_pack_job, scales));'
+        ' return 0; }\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    P = B.PackJob
+    assert got == [ctypes.sizeof(P), P.W.offset, P.N.offset, P.K.offset, P.bits.offset, P.packed.offset,
+                   P.scales.offset]
+
+
+def test_quantize_pack_many_argument_checks(L):
+    A = 0x10000          # aligned fake addresses; none of these calls gets past the checks
+    ok = (A, 4, 128, 4, A, A)
+    assert _many(L, *_jobs(ok), group=64) == B.WQ_ERR_UNSUPPORTED_GROUP
+    assert L.wq_quantize_pack_many(None, 2, 128, None) == B.WQ_ERR_INVALID_ARG
+    assert L.wq_quantize_pack_many(None, 0, 128, None) == B.WQ_OK
+    assert _many(L, _jobs(ok)[0], -1) == B.WQ_ERR_INVALID_ARG
+    assert _many(L, *_jobs(ok, (A, 4, 128, 8, A, A))) == B.WQ_ERR_UNSUPPORTED_BITS
+    assert b"job 1" in L.wq_last_error()
+    assert _many(L, *_jobs((A, 4, 128, 2, A, A), ok)) == B.WQ_ERR_UNSUPPORTED_BITS
+    assert b"job 0" in L.wq_last_error()
+    assert _many(L, *_jobs(ok, ok, (A, 4, 130, 4, A, A))) == B.WQ_ERR_INVALID_ARG
+    assert _many(L, *_jobs(ok, (A, -1, 128, 4, A, A))) == B.WQ_ERR_INVALID_ARG
+    assert _many(L, *_jobs((0, 4, 128, 4, A, A))) == B.WQ_ERR_INVALID_ARG
+    assert _many(L, *_jobs(ok, (A, 4, 128, 5, A + 8, A))) == B.WQ_ERR_MISALIGNED
+    assert _many(L, *_jobs((A, 4, 128, 6, A, A + 4))) == B.WQ_ERR_MISALIGNED
+    # a bad job after empty ones is still found; all-empty job lists need no device
+    assert _many(L, *_jobs((0, 0, 128, 4, 0, 0), (A, 4, 128, 9, A, A))) == B.WQ_ERR_UNSUPPORTED_BITS
+    assert _many(L, *_jobs((0, 0, 128, 4, 0, 0), (0, 3, 0, 7, 0, 0))) == B.WQ_OK
+
+
 def _lin(L, M=16, K=256, N=64, bits=4, group=128, rank=0, L1=0, L2=0, x=0x10000, p=0x10000,
          s=0x10000, bias=0, y=0x10000, ws=0, ws_bytes=0, path=0):
     v = ctypes.c_void_p
@@ -124,6 +172,7 @@ def test_calls_fail_cleanly_without_a_device(L):
         pass
     A = 0x10000
     assert _qp(L, A, 4, 128, 4, 128, A, A) == B.WQ_ERR_CUDA
+    assert _many(L, *_jobs((A, 4, 128, 4, A, A))) == B.WQ_ERR_CUDA
     assert _lin(L) == B.WQ_ERR_CUDA
     assert L.wq_last_error()
 

@@ -240,6 +240,64 @@ def test_model_pack_sample():
         assert snr > 3.0 * bits, (N, K, bits, snr)
 
 
+def _assert_pack_matches(packed, scales, W, bits, what=""):
+    codes, s_o = oracle.quantize(W, bits)
+    p_o = oracle.pack(codes, bits)
+    p = packed.cpu().numpy()
+    s = scales.cpu().numpy()
+    assert p.shape == p_o.shape and s.shape == s_o.shape, what
+    bad = np.argwhere(p != p_o)
+    assert bad.size == 0, f"{what}: {len(bad)} packed bytes differ, first at {bad[:4].tolist()}"
+    assert (s.view(np.uint32) == s_o.view(np.uint32)).all(), what
+
+
+def test_pack_many_parity():
+    """wq_quantize_pack_many over a shuffled job list: every width, group counts that are not
+    a multiple of a warp's 16-group block, empty jobs, 70 tensors of one width (two launches
+    of that width), planted edge groups (all-zero, ties, tiny values, outliers). Every job is
+    bit-exact against the oracle."""
+    import torch
+    rng = np.random.default_rng(777)
+    specs = [(1 + i % 5, 128 * (1 + i % 3), 5) for i in range(70)]
+    specs += [(0, 256, 4), (3, 0, 6), (7, 384, 3), (37, 1280, 4), (300, 640, 6), (1000, 2048, 7),
+              (5, 128, 3), (256, 512, 4), (33, 768, 5)]
+    jobs, host = [], []
+    for k in rng.permutation(len(specs)):
+        N, K, bits = specs[k]
+        W = edge_weight(rng, N, K, bits) if N * K else np.zeros((N, K), np.uint16)
+        host.append((W, bits))
+        jobs.append((to_dev_bf16(W), bits))
+    outs = wq.wq_quantize_pack_many(jobs)
+    torch.cuda.synchronize()
+    assert len(outs) == len(jobs)
+    for j, ((W, bits), (packed, scales)) in enumerate(zip(host, outs)):
+        _assert_pack_matches(packed, scales, W, bits, f"job {j} {W.shape} b{bits}")
+
+
+def test_pack_many_model_block():
+    """One DiT block of the whole-model workload (8 x 5120x5120, 13824x5120, 5120x13824 at
+    the mixed-precision widths, 351 M weights) through one wq_quantize_pack_many call, the
+    prepared call of the benchmark: 24 sampled rows of every tensor (first, last and random
+    ones; rows quantize independently) bit-exact against the oracle on those rows."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    widths = synth.mixed_bits(len(synth.BLOCK_SHAPES), config=5, block=3)
+    Ws = [(torch.randn(N, K, device="cuda", generator=g, dtype=torch.float32) * 0.015).to(torch.bfloat16)
+          for N, K in synth.BLOCK_SHAPES]
+    call = wq.PackJobs(list(zip(Ws, widths)))
+    call()
+    call()                                    # a second run through the same descriptors
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(11)
+    for i, (W, bits, (packed, scales)) in enumerate(zip(Ws, widths, call.outputs)):
+        N, K = W.shape
+        rows = np.unique(np.concatenate([[0, 1, N - 1], rng.integers(0, N, 21)]))
+        rows_t = torch.from_numpy(rows).cuda()
+        Wh = from_dev_bf16(W[rows_t])
+        _assert_pack_matches(packed[rows_t], scales[rows_t], Wh, bits, f"tensor {i} ({N}x{K}, b{bits})")
+
+
 # ------------------------------------------------------------------ failure detection
 
 def test_bounded_wait_selftest():
