@@ -24,7 +24,7 @@
 //   * quantize two weights per instruction with the packed fp32 pair operations of sm_100
 //     (mul/add/sub .f32x2);
 //   * codes are formed by the fp32 adder itself (see "Codes" below) and packed with shifts,
-//     byte permutes and one 16-byte (4-bit) or b 4-byte stores.
+//     byte permutes and one 16-byte (4-bit) or b 4-byte stores per lane.
 //
 // Exactness: q must equal round_half_even(fl32(w / step)). The kernel multiplies by the
 // correctly rounded reciprocal and recomputes with an IEEE division only when the product
@@ -94,10 +94,11 @@ template <int BITS>
 __host__ __device__ constexpr int pack_stage_words() { return BITS == 4 ? 1 : kPackGroupsPerWarp * 4 * BITS; }
 
 // One warp quantizes and packs the kPackGroupsPerWarp groups [g0, g0 + 16) of one tensor
-// (groups at or past n_groups are skipped). stage_w: the warp's pack_stage_words<BITS>()
-// words of shared memory (16-byte aligned), used to turn the lanes' b-word slices into
-// 16-byte stores.
-template <int BITS>
+// (groups at or past n_groups are skipped). Widths other than 4 write each lane's b words
+// either straight to memory (DIRECT: b 4-byte stores per lane, which the L2 merges into
+// whole lines) or through stage_w, the warp's pack_stage_words<BITS>() words of shared
+// memory (16-byte aligned), as 16-byte stores; the staged form needs fewer registers.
+template <int BITS, bool DIRECT>
 __device__ __forceinline__ void pack_block(const uint16_t *__restrict__ W, int64_t n_groups,
                                            uint8_t *__restrict__ packed, float *__restrict__ scales,
                                            int64_t g0, uint32_t *stage_w, int lane) {
@@ -202,12 +203,20 @@ __device__ __forceinline__ void pack_block(const uint16_t *__restrict__ W, int64
                 Nw[wd] |= T << sh;
                 if (sh + 4 * BITS > 32) Nw[wd + 1] |= T >> (32 - sh);
             }
-            uint32_t *dst = stage_w + (8 * u + gi) * 4 * BITS + l4 * BITS;
+            if constexpr (DIRECT) {
+                if (g < n_groups) {
+                    uint32_t *dst = reinterpret_cast<uint32_t *>(packed + g * kGroupBytes + l4 * 4 * BITS);
 #pragma unroll
-            for (int k = 0; k < BITS; ++k) dst[k] = __byte_perm(Nw[BITS - 1 - k], 0, 0x0123u);
+                    for (int k = 0; k < BITS; ++k) dst[k] = __byte_perm(Nw[BITS - 1 - k], 0, 0x0123u);
+                }
+            } else {
+                uint32_t *dst = stage_w + (8 * u + gi) * 4 * BITS + l4 * BITS;
+#pragma unroll
+                for (int k = 0; k < BITS; ++k) dst[k] = __byte_perm(Nw[BITS - 1 - k], 0, 0x0123u);
+            }
         }
     }
-    if constexpr (BITS != 4) {
+    if constexpr (BITS != 4 && !DIRECT) {
         __syncwarp();
         const int64_t valid = min((int64_t)GW, n_groups - g0);
         const int chunks = (int)(valid * kGroupBytes / 16);
@@ -222,12 +231,11 @@ template <int BITS>
 __global__ void __launch_bounds__(kPackThreads, 6)
 quantize_pack_kernel(const uint16_t *__restrict__ W, int64_t n_groups,
                      uint8_t *__restrict__ packed, float *__restrict__ scales) {
-    __shared__ __align__(16) uint32_t stage[kPackThreads / 32][pack_stage_words<BITS>()];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t warp_id = (int64_t)blockIdx.x * (kPackThreads / 32) + warp;
     const int64_t n_warps = (int64_t)gridDim.x * (kPackThreads / 32);
     for (int64_t g0 = warp_id * kPackGroupsPerWarp; g0 < n_groups; g0 += n_warps * kPackGroupsPerWarp)
-        pack_block<BITS>(W, n_groups, packed, scales, g0, stage[warp], lane);
+        pack_block<BITS, true>(W, n_groups, packed, scales, g0, nullptr, lane);
 }
 
 // Many tensors of one width in one launch (the mixed-precision article quantizes a whole
@@ -261,8 +269,8 @@ quantize_pack_many_kernel(const __grid_constant__ PackSegments segs) {
             const int j = base + lane;
             s += __popc(__ballot_sync(0xffffffffu, j < segs.n && segs.vbegin[j + 1] <= v0));
         }
-        pack_block<BITS>(segs.W[s], segs.n_groups[s], segs.packed[s], segs.scales[s], v0 - segs.vbegin[s],
-                         stage[warp], lane);
+        pack_block<BITS, false>(segs.W[s], segs.n_groups[s], segs.packed[s], segs.scales[s], v0 - segs.vbegin[s],
+                                stage[warp], lane);
     }
 }
 
