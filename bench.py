@@ -177,10 +177,13 @@ def run_step(wq, lins, ws, pack, events=None):
             events[2 + i].record()
 
 
-# ----------------------------------------------------------------------------- measured traffic
+# ----------------------------------------------------------------------------- recorded traffic
 
-TRAFFIC_PROFILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
-                               "wq_linear_traffic_flux3_m4096_r32.md")
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per wq_linear call of the step
+# (prepass + tensor-core kernel, mean over the 3 shapes), recorded from one ncu capture of
+# this workload, keyed by a digest of the kernel sources it was taken on; a changed kernel
+# reports null until it is captured again.
+RECORDED_TRAFFIC = {}
 KERNEL_SOURCES = ("gemm_tc.cuh", "unpack.cuh", "common.cuh", "wq_api.cu")
 
 
@@ -194,19 +197,8 @@ def kernel_source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic():
-    """DRAM bytes per wq_linear call (prepass + tensor-core kernel, mean over the 3 shapes) from
-    the committed ncu summary, or None when the kernel sources changed since it was taken."""
-    import re
-    try:
-        text = open(TRAFFIC_PROFILE).read()
-    except OSError:
-        return None
-    m_b = re.search(r"^traffic_bytes_per_call:\s*([0-9.eE+]+)", text, re.M)
-    m_h = re.search(r"^source_digest:\s*([0-9a-f]+)", text, re.M)
-    if not m_b or not m_h or m_h.group(1) != kernel_source_digest():
-        return None
-    return float(m_b.group(1))
+def recorded_traffic():
+    return RECORDED_TRAFFIC.get(kernel_source_digest())
 
 
 # ----------------------------------------------------------------------------- oracle legs
@@ -340,7 +332,9 @@ def main_arm(args):
     peaks, peak_src = load_peaks()
     lin_tflops = step_flops / (lin_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": lin_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": lin_tflops / peaks["bf16_tflops"], "traffic": measured_traffic(),
+                "frac": lin_tflops / peaks["bf16_tflops"], "traffic": recorded_traffic(),
+                "traffic_source": "recorded: ncu dram__bytes_read.sum + dram__bytes_write.sum per call, "
+                                  "same workload and kernel sources (null when the kernel changed since)",
                 "kernel": "wq_linear (lowrank_prepass_kernel + tc_linear_kernel<4>), mean over the 3 shapes",
                 "peak_source": f"{peak_src} bf16 dense (burst)"}
 
@@ -372,6 +366,8 @@ def main_arm(args):
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if world == 1 and not args.no_legs:
+        line["breakdown"].update(breakdown_legs(wq, device, peaks))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline([d["host"] for d in lins], budget_s=args.cpu_budget)
     if rank == 0:
@@ -380,6 +376,141 @@ def main_arm(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def _l2_flusher(device):
+    """Write then read a 256 MB buffer (twice the 126 MB L2) so the next call starts cold."""
+    import torch
+    flush = torch.empty(32 << 20, dtype=torch.int64, device=device)
+    sink = torch.empty((), dtype=torch.int64, device=device)
+
+    def f():
+        flush.fill_(1)
+        torch.sum(flush, dim=0, out=sink)
+    return f
+
+
+def _time_calls(run, reps, flush=None, warmup=3):
+    """Median device time (us) of `run`, each call bracketed by its own CUDA events on the
+    current stream, optionally with L2 flushed before it (outside the events)."""
+    import torch
+    for _ in range(warmup):
+        if flush:
+            flush()
+        run()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in evs:
+        if flush:
+            flush()
+        a.record()
+        run()
+        b.record()
+    torch.cuda.synchronize()
+    t = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)
+    return t[len(t) // 2]
+
+
+def breakdown_legs(wq, device, peaks, stack_blocks=40, model_blocks=49):
+    """The parts of the metric beyond the step, each timed on the device (CUDA events):
+
+    small_m     weight GB/s and HBM fraction of the Wan-like 13824x5120 and 5120x5120 linears
+                at 1 and 16 tokens, 4 and 5 bits (L2 flushed before every call);
+    m128        the 128-token crossover of the same shapes at 4 bits, against whichever
+                roofline bound binds (max of FLOPs at the bf16 peak and bytes at HBM);
+    stack       the mixed-precision 40-block DiT stack: 4096 tokens through all 400 linears in
+                order (each output is the next input), TFLOP/s of a whole pass;
+    model       whole-model quantize+pack: all 490 tensors of the 49-block model resident
+                (34.4 GB bf16), one wq_quantize_pack_many call, Gparam/s and packed size.
+    Weights are seeded device draws of the workloads' recipe."""
+    import torch
+    from bit_weight_quantization_wq_b200 import synth
+    hbm, bf16, bf16_s = peaks["hbm_gbs"], peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+    flush = _l2_flusher(device)
+    out = {}
+    # ------------------------------------------------------------ small M and the crossover
+    small, cross = [], []
+    for si, (N, K) in enumerate(synth.WAN_SHAPES):
+        for bits in (4, 5):
+            W = synth.weight_torch(synth.torch_generator(3, si, 0), N, K, 0.015)
+            packed, scales = wq.wq_quantize_pack(W, bits)
+            del W
+            b = (torch.randn(N, device=device) * 0.01).to(torch.bfloat16)
+            for M in ((1, 16, 128) if bits == 4 else (1, 16)):
+                x = torch.randn(M, K, device=device).to(torch.bfloat16)
+                y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+                us = _time_calls(lambda: wq.wq_linear(x, packed, scales, bits, N, bias=b, y=y), 30, flush)
+                wbytes = weight_bytes(N, K, bits)
+                nbytes = wbytes + 2 * M * K + 2 * M * N + 2 * N
+                flops = gemm_flops(N, K, M, 0)
+                rec = {"shape": f"{N}x{K}", "M": M, "bits": bits, "us": us,
+                       "weight_gbs": wbytes / us / 1e3, "tflops": flops / us / 1e6}
+                if M <= 16:
+                    rec["hbm_frac"] = nbytes / us / 1e3 / hbm
+                    small.append(rec)
+                else:
+                    t_roof = max(flops / (bf16 * 1e12), nbytes / (hbm * 1e9)) * 1e6
+                    rec["bound"] = "tensor" if flops / (bf16 * 1e12) > nbytes / (hbm * 1e9) else "hbm"
+                    rec["roofline_us"] = t_roof
+                    rec["frac"] = t_roof / us
+                    cross.append(rec)
+    out["small_m"] = {"l2": "flushed before every call", "peak_hbm_gbs": hbm, "cases": small}
+    out["m128"] = {"l2": "flushed before every call", "cases": cross}
+    torch.cuda.empty_cache()
+    # ------------------------------------------------------------ 40-block stack (config 4)
+    layers = []
+    for blk in range(stack_blocks):
+        widths = synth.mixed_bits(len(synth.BLOCK_SHAPES), config=4, block=blk)
+        Ws = [synth.weight_torch(synth.torch_generator(4, blk, i), N, K, 0.015)
+              for i, (N, K) in enumerate(synth.BLOCK_SHAPES)]
+        outs = wq.PackJobs(list(zip(Ws, widths)))()
+        for (N, K), bits, (p, sc) in zip(synth.BLOCK_SHAPES, widths, outs):
+            layers.append((N, K, bits, p, sc))
+        del Ws
+    Mt = 4096
+    x0 = torch.randn(Mt, 5120, device=device).to(torch.bfloat16)
+    bufs = {5120: [torch.empty((Mt, 5120), dtype=torch.bfloat16, device=device) for _ in range(2)],
+            13824: [torch.empty((Mt, 13824), dtype=torch.bfloat16, device=device)]}
+
+    def stack_pass():
+        cur, k = x0, 0
+        for N, K, bits, p, sc in layers:
+            ys = bufs[N]
+            y = ys[k % len(ys)]
+            k += 1
+            wq.wq_linear(cur, p, sc, bits, N, y=y)
+            cur = y
+
+    stack_flops = sum(gemm_flops(N, K, Mt, 0) for N, K, _, _, _ in layers)
+    us = _time_calls(stack_pass, 3, None, warmup=2)
+    tf = stack_flops / us / 1e6
+    out["stack"] = {"blocks": stack_blocks, "linears": len(layers), "tokens": Mt, "ms_per_pass": us / 1e3,
+                    "tflops": tf, "frac_bf16_sustained": tf / bf16_s, "frac_bf16_burst": tf / bf16,
+                    "bits_histogram": {str(b): sum(1 for l in layers if l[2] == b) for b in range(3, 8)},
+                    "l2": "inputs larger than L2 (8.8 GB of packed weights per pass)"}
+    del layers, bufs, x0
+    torch.cuda.empty_cache()
+    # ------------------------------------------------------------ 49-block model pack (config 5)
+    jobs = []
+    for blk in range(model_blocks):
+        widths = synth.mixed_bits(len(synth.BLOCK_SHAPES), config=5, block=blk)
+        for i, ((N, K), bits) in enumerate(zip(synth.BLOCK_SHAPES, widths)):
+            jobs.append((synth.weight_torch(synth.torch_generator(5, blk, i), N, K, 0.015), bits))
+    call = wq.PackJobs(jobs)
+    l0 = wq.wq_launch_count()
+    call()
+    launches = wq.wq_launch_count() - l0
+    us = _time_calls(call, 5, None, warmup=2)
+    params = sum(W.numel() for W, _ in jobs)
+    packed_b = sum(p.numel() + 4 * sc.numel() for p, sc in call.outputs)
+    nbytes = 2 * params + packed_b
+    out["model"] = {"blocks": model_blocks, "tensors": len(jobs), "params": params, "ms_per_call": us / 1e3,
+                    "gparams": params / us / 1e3, "gbs": nbytes / us / 1e3, "hbm_frac": nbytes / us / 1e3 / hbm,
+                    "bf16_gb": 2 * params / 1e9, "packed_gb": packed_b / 1e9, "launches_per_call": launches,
+                    "l2": "inputs larger than L2 (34 GB of weights per call)"}
+    del jobs, call
+    torch.cuda.empty_cache()
+    return out
 
 
 def e2e_leg(wq, lins, ws, args, device, world, step_flops):
@@ -579,6 +710,7 @@ def parse(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-legs", action="store_true", help="skip the small-M / crossover / stack / model legs")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--case", default=None,
                     help="time one shape: pack:N,K,bits, linear:M,N,K,bits,rank, model:BLOCKS or model_per_tensor:BLOCKS")

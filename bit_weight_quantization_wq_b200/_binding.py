@@ -63,7 +63,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         i64, i32, sz, p = ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
         L.wq_version.argtypes, L.wq_version.restype = [], i32
-        L.wq_packed_bytes.argtypes, L.wq_packed_bytes.restype = [i64, i64, i32], sz
+        L.wq_packed_bytes.argtypes, L.wq_packed_bytes.restype = [i64, i64, i32, i32], sz
         L.wq_scales_count.argtypes, L.wq_scales_count.restype = [i64, i64, i32], i64
         L.wq_quantize_pack.argtypes = [p, i64, i64, i32, i32, p, p, p]
         L.wq_quantize_pack.restype = i32
@@ -128,8 +128,8 @@ def wq_version() -> int:
     return int(lib().wq_version())
 
 
-def wq_packed_bytes(N: int, K: int, bits: int) -> int:
-    return int(lib().wq_packed_bytes(N, K, bits))
+def wq_packed_bytes(N: int, K: int, bits: int, group: int = 128) -> int:
+    return int(lib().wq_packed_bytes(N, K, bits, group))
 
 
 def wq_scales_count(N: int, K: int, group: int = 128) -> int:

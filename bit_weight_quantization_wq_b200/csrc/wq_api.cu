@@ -73,6 +73,20 @@ wq_status current_device(int *dev_out, const DeviceInfo **info) {
 
 std::atomic<uint64_t> g_launches{0};
 
+// One-time per-device set-up (kernel attributes) that concurrent host threads may race to:
+// the first caller runs f() under a mutex, later callers see the flag and skip it. A failed
+// set-up is retried by the next call.
+std::mutex g_setup_mutex;
+template <class F>
+cudaError_t setup_once(std::atomic<int> (&done)[kMaxDevices], int dev, F &&f) {
+    if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    if (done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+    const cudaError_t e = f();
+    if (e == cudaSuccess) done[dev].store(1, std::memory_order_release);
+    return e;
+}
+
 // Called right after every kernel launch: counts it and reports a launch error.
 wq_status check_launch(const char *what) {
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -173,9 +187,11 @@ bool small_layout(int bits, int rows, int gcta, bool even, bool scale_tma, int s
 // Clusters of S CTAs that fit at once (one CTA per SM, the most shared memory), cached.
 template <int BITS, int TOK>
 int small_max_clusters(int dev, int S, int sm_count) {
-    static int cache[kMaxDevices][3] = {};
+    // computed once per device and cluster size; two threads racing here compute the same value
+    static std::atomic<int> cache[kMaxDevices][3] = {};
     const int si = S == 1 ? 0 : (S == 2 ? 1 : 2);
-    if (cache[dev][si] != 0) return cache[dev][si];
+    const int cached = cache[dev][si].load(std::memory_order_relaxed);
+    if (cached != 0) return cached;
     int n = sm_count / S;
     if (S > 1) {
         cudaLaunchConfig_t cfg = {};
@@ -194,8 +210,9 @@ int small_max_clusters(int dev, int S, int sm_count) {
         cudaGetLastError();
         n = std::min(n, q);
     }
-    cache[dev][si] = n > 0 ? n : -1;
-    return cache[dev][si];
+    const int v = n > 0 ? n : -1;
+    cache[dev][si].store(v, std::memory_order_relaxed);
+    return v;
 }
 
 wq_status get_encoder();
@@ -207,13 +224,12 @@ wq_status make_map_3d(CUtensorMap *map, CUtensorMapDataType dt, const void *base
 template <int BITS, int TOK>
 wq_status launch_smallm_tok(wq::SmallMArgs a, const uint8_t *packed, int dev, int sm_count, cudaStream_t st) {
     using T = wq::SmTok<TOK>;
-    static bool attr_done[kMaxDevices] = {};
-    if (!attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(wq::smallm_kernel<BITS, TOK>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smallm)");
-        attr_done[dev] = true;
-    }
+    static std::atomic<int> attr_done[kMaxDevices] = {};
+    cudaError_t e = setup_once(attr_done, dev, [] {
+        return cudaFuncSetAttribute(wq::smallm_kernel<BITS, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSmemMax);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smallm)");
     const int64_t U = (a.N + 15) / 16;
     const int G = (int)(a.K / 128);
     // cluster size S (K split) and cluster count C: the fewest items on the busiest CTA,
@@ -285,8 +301,7 @@ wq_status launch_smallm_tok(wq::SmallMArgs a, const uint8_t *packed, int dev, in
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = bestS > 1 ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, wq::smallm_kernel<BITS, TOK>, pm64, pm32, pm16, pm_tail, xm_full, xm_tail,
-                                       sm_map, a);
+    e = cudaLaunchKernelEx(&cfg, wq::smallm_kernel<BITS, TOK>, pm64, pm32, pm16, pm_tail, xm_full, xm_tail, sm_map, a);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(smallm_kernel)");
     return check_launch("smallm_kernel");
 }
@@ -380,15 +395,14 @@ template <int BITS>
 wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &pm, const CUtensorMap &tm,
                     const CUtensorMap &lm, int l_tma, int sm_count, cudaStream_t st) {
     using L = wq::TcLayout<BITS>;
-    static bool attr_done[kMaxDevices] = {};
+    static std::atomic<int> attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(wq::tc_linear_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)L::kAlloc);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc_linear_kernel)");
-        attr_done[dev] = true;
-    }
+    const cudaError_t e = setup_once(attr_done, dev, [] {
+        return cudaFuncSetAttribute(wq::tc_linear_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)L::kAlloc);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc_linear_kernel)");
     wq::TcParams p{};
     p.scales = a.scales;
     p.L2 = static_cast<const uint16_t *>(a.L2);
@@ -411,15 +425,13 @@ wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_
     // The prepass is latency-bound (each CTA walks its K share one 64-k block at a time), so
     // K is split (clusters of up to 16 CTAs, a non-portable size) until about eight CTAs per
     // SM are in flight.
-    static bool attr_done[kMaxDevices] = {};
+    static std::atomic<int> attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(wq::lowrank_prepass_kernel<R>,
-                                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(lowrank_prepass_kernel)");
-        attr_done[dev] = true;
-    }
+    cudaError_t e = setup_once(attr_done, dev, [] {
+        return cudaFuncSetAttribute(wq::lowrank_prepass_kernel<R>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(lowrank_prepass_kernel)");
     const int kmax = 16;
     int ks = 1;
     while (ks < kmax && ks * 2 <= nkb && mtiles * ks < 8 * (int64_t)sm_count) ks *= 2;
@@ -435,7 +447,7 @@ wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, wq::lowrank_prepass_kernel<R>, static_cast<const uint16_t *>(a.x),
+    e = cudaLaunchKernelEx(&cfg, wq::lowrank_prepass_kernel<R>, static_cast<const uint16_t *>(a.x),
                                        static_cast<const uint16_t *>(a.L1), t, a.M, a.K);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(lowrank_prepass_kernel)");
     return check_launch("lowrank_prepass_kernel");
@@ -515,8 +527,8 @@ extern "C" {
 
 int wq_version(void) { return 100; }
 
-size_t wq_packed_bytes(int64_t N, int64_t K, int bits) {
-    if (N < 0 || K < 0 || bits < 3 || bits > 7 || (K * bits) % 8 != 0) return 0;
+size_t wq_packed_bytes(int64_t N, int64_t K, int bits, int group) {
+    if (N < 0 || K < 0 || bits < 3 || bits > 7 || group != 128 || K % group != 0) return 0;
     return (size_t)N * (size_t)K * (size_t)bits / 8;
 }
 

@@ -79,6 +79,30 @@ def bias(rng: np.random.Generator, N: int, sigma: float = 0.01) -> np.ndarray:
     return f32_to_bf16_bits(rng.standard_normal(N, dtype=np.float32) * np.float32(sigma))
 
 
+def torch_generator(config: int, block: int = 0, idx: int = 0, device="cuda"):
+    """A torch generator on `device` seeded from (config, block, tensor index), for the
+    workloads too large to draw on the host (the 40-block stack and the 49-block model)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(((1000 + config) * 1_000_003 + block) * 1009 + idx)
+    return g
+
+
+def weight_torch(gen, N: int, K: int, sigma: float, outlier_frac: float = 1e-3, device="cuda"):
+    """The :func:`weight` recipe drawn with a torch generator on the device: N x K bf16 torch
+    tensor, N(0, sigma^2) body with round(outlier_frac * N * K) distinct outlier positions,
+    each +-1 (p = 1/2) times U(0.2, 0.5); fp32 draws rounded to bf16 (nearest even)."""
+    import torch
+    w = torch.randn(N, K, device=device, generator=gen, dtype=torch.float32) * sigma
+    n_out = int(round(outlier_frac * N * K))
+    if n_out:
+        pos = torch.randperm(N * K, device=device, generator=gen)[:n_out]
+        sign = torch.where(torch.rand(n_out, device=device, generator=gen) < 0.5, -1.0, 1.0)
+        mag = torch.rand(n_out, device=device, generator=gen, dtype=torch.float64) * 0.3 + 0.2
+        w.view(-1)[pos] = (sign * mag).to(torch.float32)
+    return w.to(torch.bfloat16)
+
+
 def lowrank_split(W_bits: np.ndarray, rank: int, rng: np.random.Generator, power_iters: int = 4):
     """Split W into a rank-r bf16 branch and a bf16 residual, as an SVDQuant model ships it.
 

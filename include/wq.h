@@ -69,10 +69,11 @@ typedef enum {
 /* Library version, as 10000*major + 100*minor + patch. */
 WQ_API int wq_version(void);
 
-/* Bytes of the packed codes of an N x K weight at `bits` bits: N * K * bits / 8
- * ([PG] sec. 3.3 packing table: every 128-weight group takes 16*bits bytes).
- * Returns 0 when the arguments are invalid. */
-WQ_API size_t wq_packed_bytes(int64_t N, int64_t K, int bits);
+/* Bytes of the packed codes of an N x K weight at `bits` bits with groups of `group`
+ * input weights: N * K * bits / 8 ([PG] sec. 3.3 packing table: every 128-weight group
+ * takes 16*bits bytes). Returns 0 when the arguments are invalid: bits outside 3..7,
+ * group != 128, a negative size, or K not a multiple of the group. */
+WQ_API size_t wq_packed_bytes(int64_t N, int64_t K, int bits, int group);
 
 /* Number of fp32 scales of an N x K weight: N * K / group ([PG] sec. 3.1: one step per
  * group of `group` consecutive input weights). Returns -1 when invalid. */

@@ -16,7 +16,7 @@
  *          W = (16-bit low-rank branch) + (4-bit residual), so the layer output is
  *          x * deq(R)^T + x * L1 * L2.
  *
- * Readings taken where the pages leave a step open (listed again in the design doc):
+ * Readings taken where the pages leave a step open:
  *   - all quantizer arithmetic is IEEE fp32, round-to-nearest-even, no FMA contraction;
  *     1.01 is rounded to fp32 before the multiply;
  *   - round() is round-half-to-even;

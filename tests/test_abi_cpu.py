@@ -39,6 +39,75 @@ def test_exports_match_header(L):
         assert hasattr(L, name)
 
 
+# The boundary calls as the hot-path scope lists them (argument types in order, return
+# type), checked against the header by the C compiler. Two deliberate differences from
+# that list: wq_linear_workspace_bytes also takes the low-rank `rank` (only the branch
+# needs scratch, so the size depends on it), and the device status is read with
+# wq_device_status(stream, clear).
+SCOPE_SIGNATURES = {
+    "wq_packed_bytes": "size_t (*)(int64_t, int64_t, int, int)",
+    "wq_scales_count": "int64_t (*)(int64_t, int64_t, int)",
+    "wq_quantize_pack": "wq_status (*)(const void *, int64_t, int64_t, int, int, uint8_t *, float *, wq_stream_t)",
+    "wq_linear_workspace_bytes": "size_t (*)(int64_t, int64_t, int64_t, int, int)",
+    "wq_linear": ("wq_status (*)(const void *, int64_t, int64_t, const uint8_t *, const float *, int, int, int64_t, "
+                  "const void *, const void *, int, const void *, void *, void *, size_t, wq_stream_t)"),
+    "wq_status_string": "const char *(*)(wq_status)",
+}
+
+
+def test_scope_signatures_match_header(tmp_path):
+    """Every boundary call of the hot-path scope has exactly the expected C signature."""
+    checks = "\n".join(
+        f'_Static_assert(_Generic(&{name}, {sig}: 1, default: 0), "{name} signature");'
+        for name, sig in SCOPE_SIGNATURES.items())
+    src = tmp_path / "sig.c"
+    src.write_text('#include "wq.h"\n' + checks + "\nint main(void) { return 0; }\n")
+    r = subprocess.run(["gcc", "-std=c11", "-fsyntax-only", "-I", os.path.join(ROOT, "include"), str(src)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
+_CTYPES = {"int64_t": ctypes.c_int64, "int": ctypes.c_int, "size_t": ctypes.c_size_t,
+           "uint32_t": ctypes.c_uint32, "uint64_t": ctypes.c_uint64, "wq_status": ctypes.c_int,
+           "wq_path": ctypes.c_int, "wq_stream_t": ctypes.c_void_p}
+
+
+def _ctype_of(decl):
+    decl = decl.replace("const ", "").strip()
+    if decl in ("void", ""):
+        return None
+    if decl.startswith("char") and "*" in decl:
+        return ctypes.c_char_p
+    if "*" in decl:
+        base = decl.split("*")[0].strip()
+        return ctypes.POINTER(B.PackJob) if base == "wq_pack_job" else ctypes.c_void_p
+    return _CTYPES[decl.split()[0]]
+
+
+def header_prototypes():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for ret, name, args in re.findall(r"WQ_API\s+([\w\s\*]+?)\s*\b(wq_\w+)\s*\(([^)]*)\)", text):
+        params = [a.strip() for a in args.split(",") if a.strip() and a.strip() != "void"]
+        # drop the parameter name: the type is everything before the last identifier
+        types = [re.sub(r"\b\w+\s*$", "", p).strip() or p for p in params]
+        out[name] = (ret.strip(), types)
+    return out
+
+
+def test_binding_declarations_match_header(L):
+    """The binding's ctypes argtypes/restype follow the header's prototypes, call by call."""
+    protos = header_prototypes()
+    assert sorted(protos) == sorted(B.SYMBOLS)
+    for name, (ret, types) in protos.items():
+        f = getattr(L, name)
+        want = [_ctype_of(t) for t in types]
+        assert list(f.argtypes) == want, (name, f.argtypes, want)
+        r = _ctype_of(ret)
+        if r is not None:
+            assert f.restype == r, (name, f.restype, r)
+
+
 def test_no_driver_or_shared_cudart_dependency(L):
     out = subprocess.run(["ldd", B.LIB_PATH], capture_output=True, text=True, check=True).stdout
     assert "libcuda.so" not in out and "libcudart" not in out
@@ -47,10 +116,12 @@ def test_no_driver_or_shared_cudart_dependency(L):
 def test_sizes(L):
     # packing table: 16*b bytes per 128-weight group
     for bits in (3, 4, 5, 6, 7):
-        assert wq.wq_packed_bytes(5120, 5120, bits) == 5120 * 5120 * bits // 8
-        assert wq.wq_packed_bytes(1, 128, bits) == 16 * bits
-    assert wq.wq_packed_bytes(4, 128, 2) == 0 and wq.wq_packed_bytes(4, 128, 8) == 0
-    assert wq.wq_packed_bytes(-1, 128, 4) == 0
+        assert wq.wq_packed_bytes(5120, 5120, bits, 128) == 5120 * 5120 * bits // 8
+        assert wq.wq_packed_bytes(1, 128, bits, 128) == 16 * bits
+    assert wq.wq_packed_bytes(4, 128, 2, 128) == 0 and wq.wq_packed_bytes(4, 128, 8, 128) == 0
+    assert wq.wq_packed_bytes(-1, 128, 4, 128) == 0
+    assert wq.wq_packed_bytes(4, 128, 4, 64) == 0          # only groups of 128
+    assert wq.wq_packed_bytes(4, 200, 4, 128) == 0         # K not a multiple of the group
     assert wq.wq_scales_count(13824, 5120, 128) == 13824 * 40
     assert wq.wq_scales_count(3, 100, 128) == -1
     assert wq.wq_linear_workspace_bytes(16, 256, 512, 4, 0) == 0
@@ -74,12 +145,13 @@ def test_quantize_pack_argument_checks(L):
     assert _qp(L, A, 4, 128, 2, 128, A, A) == B.WQ_ERR_UNSUPPORTED_BITS
     assert _qp(L, A, 4, 128, 8, 128, A, A) == B.WQ_ERR_UNSUPPORTED_BITS
     assert _qp(L, A, 4, 128, 4, 64, A, A) == B.WQ_ERR_UNSUPPORTED_GROUP
-    assert _qp(L, A, 4, 130, 4, 128, A, A) == B.WQ_ERR_INVALID_ARG
     assert _qp(L, A, -1, 128, 4, 128, A, A) == B.WQ_ERR_INVALID_ARG
     assert _qp(L, 0, 4, 128, 4, 128, A, A) == B.WQ_ERR_INVALID_ARG
+    assert _qp(L, A, 4, 130, 4, 128, A, A) == B.WQ_ERR_INVALID_ARG
+    assert b"multiple of 128" in L.wq_last_error()
     assert _qp(L, A + 8, 4, 128, 4, 128, A, A) == B.WQ_ERR_MISALIGNED
     assert _qp(L, A, 4, 128, 4, 128, A + 4, A) == B.WQ_ERR_MISALIGNED
-    assert b"multiple of 128" in L.wq_last_error() or True
+    assert b"16-byte aligned" in L.wq_last_error()
     # empty weights are a no-op that needs no device
     assert _qp(L, 0, 0, 128, 4, 128, 0, 0) == B.WQ_OK
 

@@ -3,10 +3,12 @@ memory when they run it. The low-rank branch's scratch then comes from a buffer 
 into the library instead of a caller workspace.
 
 Checked through the C ABI (ctypes, raw device pointers): two calls in a row on each kernel
-family give the same result as wq_linear with its own workspace (within the GEMM tolerance
-of the parity tests), and a size whose scratch exceeds the static buffer is refused before
-anything runs. This file is collected last so that a run that stops at the first failure
-has already run every other test.
+family give bit for bit the result of wq_linear with its own workspace (the same kernels
+run in the same order, only the scratch address differs), the first of them is also
+compared with the CPU oracle within the GEMM tolerance of the parity tests, and a size
+whose scratch exceeds the static buffer is refused before anything runs. This file is
+collected last so that a run that stops at the first failure has already run every other
+test.
 """
 import ctypes
 
@@ -16,7 +18,8 @@ import pytest
 import bit_weight_quantization_wq_b200 as wq
 from bit_weight_quantization_wq_b200 import _binding as B
 from bit_weight_quantization_wq_b200 import synth
-from helpers import MAX_ABS_RMS, REL_FRO, bf16_f64, from_dev_bf16, to_dev_bf16
+import oracle
+from helpers import assert_linear_close, from_dev_bf16, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -52,17 +55,19 @@ def test_matches_workspace_call_twice(M, N, K, bits, rank):
     packed, scales = wq.wq_quantize_pack(to_dev_bf16(W), bits)
     ref = wq.wq_linear(x, packed, scales, bits, N, L1=L1, L2=L2, bias=b)
     torch.cuda.synchronize()
-    ref64 = bf16_f64(from_dev_bf16(ref))
-    rms = np.sqrt(np.mean(ref64 ** 2))
-    for _ in range(2):
+    ref_bits = from_dev_bf16(ref)
+    for call in range(2):
         y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         st = _call_no_workspace(x, packed, scales, bits, N, L1, L2, b, y)
         assert st == B.WQ_OK, B.lib().wq_last_error().decode()
         torch.cuda.synchronize()
-        got = bf16_f64(from_dev_bf16(y))
-        err = got - ref64
-        assert np.linalg.norm(err) / np.linalg.norm(ref64) <= REL_FRO
-        assert np.abs(err).max() <= MAX_ABS_RMS * rms
+        got = from_dev_bf16(y)
+        assert np.array_equal(got, ref_bits), f"call {call}: {int((got != ref_bits).sum())} outputs differ"
+        if call == 0:
+            codes, s_o = oracle.quantize(W, bits)
+            h = lambda t: None if t is None else from_dev_bf16(t)
+            y_o = oracle.linear_rows(from_dev_bf16(x), oracle.dequant(codes, s_o, bits), h(L1), h(L2), h(b))
+            assert_linear_close(got, y_o, f"no-workspace {M}x{N}x{K} b{bits} r{rank}")
     assert wq.wq_device_status() == 0
 
 
