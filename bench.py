@@ -421,8 +421,11 @@ def breakdown_legs(wq, device, peaks, stack_blocks=40, model_blocks=49):
     stack       the mixed-precision 40-block DiT stack: 4096 tokens through all 400 linears in
                 order (each output is the next input), TFLOP/s of a whole pass;
     model       whole-model quantize+pack: all 490 tensors of the 49-block model resident
-                (34.4 GB bf16), one wq_quantize_pack_many call, Gparam/s and packed size.
+                (34.4 GB bf16), one wq_quantize_pack_many call, Gparam/s and packed size; the
+                error table of all of them at every width (wq_quant_error_many), each tensor's
+                SNR at its width, and the per-tensor width search at 5.0 bits per weight.
     Weights are seeded device draws of the workloads' recipe."""
+    import numpy as np
     import torch
     from bit_weight_quantization_wq_b200 import synth
     hbm, bf16, bf16_s = peaks["hbm_gbs"], peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
@@ -508,7 +511,29 @@ def breakdown_legs(wq, device, peaks, stack_blocks=40, model_blocks=49):
                     "gparams": params / us / 1e3, "gbs": nbytes / us / 1e3, "hbm_frac": nbytes / us / 1e3 / hbm,
                     "bf16_gb": 2 * params / 1e9, "packed_gb": packed_b / 1e9, "launches_per_call": launches,
                     "l2": "inputs larger than L2 (34 GB of weights per call)"}
-    del jobs, call
+    # error table of all 490 tensors at every width (one wq_quant_error_many call), each
+    # tensor's SNR at its width, and the per-tensor width search at 5.0 bits per weight
+    Ws = [W for W, _ in jobs]
+    widths = np.array([b for _, b in jobs])
+    table = torch.empty((len(Ws), 6), dtype=torch.float64, device=device)
+    err_call = lambda: wq.wq_quant_error_many(Ws, out=table)
+    us_err = _time_calls(err_call, 3, None, warmup=1)
+    tab = table.cpu().numpy()
+    n_w = np.array([W.numel() for W in Ws], np.int64)
+    sse_at = tab[np.arange(len(Ws)), widths - 3]
+    snr = 10.0 * np.log10(tab[:, 5] / sse_at)
+    mse = tab[:, :5] / n_w[:, None]
+    t_init = np.random.default_rng(5).standard_normal((15, len(Ws))) * 0.5
+    pd_bits, pd_mse, pd_bpw, _ = wq.wq_pd_search(mse, n_w, [3, 4, 5, 6, 7], 5.0, t_init)
+    tot = lambda b: float(np.sum(n_w * mse[np.arange(len(Ws)), np.asarray(b) - 3]) / n_w.sum())
+    out["model"].update({
+        "snr_db": {"mean": float(snr.mean()), "min": float(snr.min()), "max": float(snr.max()),
+                   "by_bits": {str(b): float(snr[widths == b].mean()) for b in range(3, 8) if (widths == b).any()}},
+        "error_table_ms": us_err / 1e3, "error_table_gparams": params / us_err / 1e3,
+        "pd_search_5bpw": {"bpw": pd_bpw, "mse": pd_mse, "mse_uniform_5": tot(np.full(len(Ws), 5)),
+                           "mse_histogram_widths": tot(widths),
+                           "histogram": {str(b): int((pd_bits == b).sum()) for b in range(3, 8)}}})
+    del jobs, call, Ws, table
     torch.cuda.empty_cache()
     return out
 

@@ -12,11 +12,15 @@ from ._binding import (  # noqa: F401
     WQError,
     lib,
     status_string,
+    wq_dequantize,
     wq_device_status,
     wq_launch_count,
     wq_linear,
     wq_linear_workspace_bytes,
     wq_packed_bytes,
+    wq_pd_search,
+    wq_quant_error,
+    wq_quant_error_many,
     wq_quantize_pack,
     wq_quantize_pack_many,
     wq_scales_count,

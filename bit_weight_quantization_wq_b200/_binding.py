@@ -30,7 +30,8 @@ SYMBOLS = (
     "wq_version", "wq_packed_bytes", "wq_scales_count", "wq_quantize_pack",
     "wq_linear_workspace_bytes", "wq_linear", "wq_linear_ex", "wq_device_status",
     "wq_selftest_bounded_wait", "wq_status_string", "wq_last_error", "wq_launch_count",
-    "wq_linear_no_workspace", "wq_quantize_pack_many",
+    "wq_linear_no_workspace", "wq_quantize_pack_many", "wq_quant_error", "wq_quant_error_many",
+    "wq_pd_search", "wq_dequantize",
 )
 
 
@@ -41,6 +42,11 @@ class WQError(RuntimeError):
         if detail:
             msg += f": {detail}"
         super().__init__(msg)
+
+
+class ErrorJob(ctypes.Structure):
+    """wq_error_job of include/wq.h."""
+    _fields_ = [("W", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("out", ctypes.c_void_p)]
 
 
 class PackJob(ctypes.Structure):
@@ -83,6 +89,14 @@ def lib() -> ctypes.CDLL:
         L.wq_linear_no_workspace.restype = i32
         L.wq_quantize_pack_many.argtypes = [ctypes.POINTER(PackJob), i32, i32, p]
         L.wq_quantize_pack_many.restype = i32
+        L.wq_quant_error.argtypes = [p, i64, i64, i32, p, p]
+        L.wq_quant_error.restype = i32
+        L.wq_quant_error_many.argtypes = [ctypes.POINTER(ErrorJob), i32, i32, p]
+        L.wq_quant_error_many.restype = i32
+        L.wq_pd_search.argtypes = [p, p, i32, p, i32, ctypes.c_double, i32, i32, p, p, p]
+        L.wq_pd_search.restype = i32
+        L.wq_dequantize.argtypes = [p, p, i64, i64, i32, i32, p, p]
+        L.wq_dequantize.restype = i32
         _lib = L
     return _lib
 
@@ -255,3 +269,71 @@ def wq_quantize_pack_many(jobs, group: int = 128, stream=None):
     """Quantize + pack many (N, K) bf16 weights, each at its own width, in a few launches.
     ``jobs`` as for :class:`PackJobs`. Returns one ``(packed, scales)`` per job."""
     return PackJobs(jobs, group)(stream)
+
+
+ERROR_WIDTHS = (3, 4, 5, 6, 7)
+
+
+def wq_quant_error_many(weights, group: int = 128, out=None, stream=None):
+    """Quantization error table of many (N, K) bf16 weights: a float64 CUDA tensor (T, 6) whose
+    row i holds sum (w - deq_b(w))^2 for b = 3..7 and sum w^2 of weight i."""
+    import torch
+    weights = list(weights)
+    if out is None:
+        dev = weights[0].device if weights else torch.device("cuda")
+        out = torch.empty((len(weights), 6), dtype=torch.float64, device=dev)
+    _dev(out, "out", torch.float64, (len(weights), 6))
+    descs = []
+    for i, W in enumerate(weights):
+        _dev(W, f"weights[{i}]", torch.bfloat16)
+        if W.dim() != 2:
+            raise ValueError(f"weights[{i}] must be 2-D (N, K)")
+        descs.append(ErrorJob(W.data_ptr(), W.shape[0], W.shape[1], out[i].data_ptr()))
+    arr = (ErrorJob * max(1, len(descs)))(*descs)
+    _check(lib().wq_quant_error_many(arr, len(descs), group, _stream(stream)), "wq_quant_error_many")
+    return out
+
+
+def wq_quant_error(W, group: int = 128, stream=None):
+    """Quantization error table of one (N, K) bf16 weight: float64 CUDA tensor (6,)."""
+    import torch
+    _dev(W, "W", torch.bfloat16)
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D (N, K)")
+    out = torch.empty(6, dtype=torch.float64, device=W.device)
+    _check(lib().wq_quant_error(_ptr(W), W.shape[0], W.shape[1], group, _ptr(out), _stream(stream)),
+           "wq_quant_error")
+    return out
+
+
+def wq_pd_search(mse_table, n_params, bits, target_bpw: float, t_init, n_iters: int = 500):
+    """Per-tensor width search (host). mse_table (T, B) per-weight MSE, n_params (T,), bits (B,),
+    t_init (R, T) random starts. Returns (widths int array (T,), total MSE, BPW, start index)."""
+    import numpy as np
+    mse = np.ascontiguousarray(mse_table, np.float64)
+    n = np.ascontiguousarray(n_params, np.int64)
+    b = np.ascontiguousarray(bits, np.int32)
+    t0 = np.ascontiguousarray(t_init, np.float64)
+    T, nb = mse.shape
+    if n.shape != (T,) or b.shape != (nb,) or t0.ndim != 2 or t0.shape[1] != T:
+        raise ValueError("mse_table (T, B), n_params (T,), bits (B,), t_init (R, T)")
+    out = np.empty(T, np.int32)
+    res = np.empty(3, np.float64)
+    ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    _check(lib().wq_pd_search(ptr(mse), ptr(n), T, ptr(b), nb, float(target_bpw), n_iters, t0.shape[0], ptr(t0),
+                              ptr(out), ptr(res)), "wq_pd_search")
+    return out, float(res[0]), float(res[1]), int(res[2])
+
+
+def wq_dequantize(packed, scales, bits: int, K: int, group: int = 128, out=None, stream=None):
+    """bf16 (N, K) weight bf16(q * step) from packed codes and steps (the page's dequantize)."""
+    import torch
+    _dev(packed, "packed", torch.uint8)
+    _dev(scales, "scales", torch.float32)
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device=packed.device)
+    _dev(out, "out", torch.bfloat16, (N, K))
+    _check(lib().wq_dequantize(_ptr(packed), _ptr(scales), N, K, bits, group, _ptr(out), _stream(stream)),
+           "wq_dequantize")
+    return out

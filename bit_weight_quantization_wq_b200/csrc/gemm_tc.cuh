@@ -14,30 +14,34 @@
 //
 // Orientation: D = W_q x^T, so TMEM lanes are weight rows and columns are tokens; the
 // per-group step is then one scalar per lane.
-// One persistent CTA per SM walks 128 x 128 tiles (128 weight rows x 128 tokens).
-// TMEM (512 columns): T0, T1 = per-group partials (double-buffered, 128 columns each) and
-// 8 stages of codes (32 columns = 64 k each).
-// Warp roles (512 threads):
-//   warp 0      TMA producer of x tiles (128 tokens x 64 k bf16, 128B swizzle, 16 KB/stage)
-//   warps 1, 3  warp 1 allocates TMEM; one thread of each issues tcgen05.mma (A = codes from
-//               TMEM, B = x from shared memory, M=128 N=128 K=16) for alternate units
-//   warp 2      TMA producer of packed-weight tiles (128 rows x one group, 16*b bytes a row)
-//   warps 4-7   unpack: one weight row per thread; bf16 pairs of exact q written to the A
-//               stage with tcgen05.st
+// One persistent CTA per SM walks tiles of 128 weight rows x TT tokens (TT = 256, or 128 for
+// few tokens), weight tiles fastest, so a wave of CTAs shares one token tile of x in L2 and
+// the (4-8x smaller) packed weight stays L2-resident across token tiles.
+// Shared memory: a ring of kStages 64-k stages, each holding the x tile (TT tokens x 64 k,
+// bf16, 128-byte swizzle, by TMA) and the code tile (128 rows x 64 k exact bf16 q, the same
+// swizzled layout, written by the unpack warps). TMEM (512 columns): T0, T1 = the per-group
+// partial products (double-buffered, TT columns each).
+// One unit = one 128-k group (two stages) or the low-rank unit. Per unit, one MMA-issuing
+// thread waits for T to be free and for each stage to be full, issues M=128 N=TT K=16 MMAs
+// (A = codes, B = x, both from shared memory), releases each stage with a commit and hands T
+// to the promotion with another. With TT = 256 one unit is ~1100 tensor cycles, long enough
+// to hide the promotion's hand-off of the other T buffer.
+// Warp roles (512 threads; registers re-split per warpgroup with setmaxnreg, 48/96/184,
+// summing to the 128 per thread the block is launched with):
+//   warp 0      TMA producer of the x tiles (and of t = x L1 for the low-rank unit)
+//   warps 1, 3  warp 1 allocates TMEM; one thread of each issues the MMAs of alternate units
+//   warp 2      TMA producer of the tile's [rank][128] block of L2 (when N % 8 == 0)
+//   warps 4-7   unpack: one weight row per thread, packed group straight from global memory
+//               (two groups in flight in registers) to exact bf16 q pairs in the code tile
 //   warps 8-15  promotion: R += step * T per group (fp32, two lanes per instruction) with R in
-//               registers (two warps per TMEM lane quarter, 64 columns each), then the epilogue
-//               (+ bias, round once to bf16, store y)
-// Synchronization is per unit (one 128-k group, or the low-rank unit), not per k stage: the
-// single MMA-issuing thread pays ~140 cycles per mbarrier wait, so it waits once per unit on
-// ready[slot], which completes when the unit's x tiles have landed (TMA transaction bytes),
-// its codes are in TMEM (4 unpack warps) and its T buffer is free (8 promotion warps); one
-// commit per unit releases the slot (consumed[slot]) and another hands T to the promotion.
+//               registers (two warps per TMEM lane quarter, TT/2 columns each), then the
+//               epilogue (+ bias, round once to bf16, store y)
 // Low-rank branch: one more unit per tile with B = [t_hi | t_lo] (t = x L1 split into two
-// bf16 terms by lowrank_prepass_kernel) and A = [L2^T | L2^T] (bf16 from global), promoted
-// with scale 1 into the same R; the split keeps t's rounding out of the result.
+// bf16 terms by lowrank_prepass_kernel) and A = [L2^T | L2^T], promoted with scale 1 into the
+// same R; the split keeps t's rounding out of the result.
 //
-// Every wait is bounded (see common.cuh). On a timeout the roles stop, the producer waits
-// (bounded) for its copies in flight, the MMA thread for its MMAs, and TMEM is freed.
+// Every wait is bounded (see common.cuh). On a timeout the roles stop, the producers wait
+// (bounded) for their copies in flight, the MMA threads for their MMAs, and TMEM is freed.
 #pragma once
 
 #include <cuda.h>
@@ -48,43 +52,40 @@
 namespace wq {
 
 constexpr int kTcBW = 128;                // weight rows per tile (MMA M)
-constexpr int kTcBT = 128;                // tokens per tile (MMA N)
-constexpr int kTcBK = 64;                 // k per x stage / A stage
-constexpr int kTcSlots = 4;               // units in flight (each: 2 x stages + 2 code stages)
-constexpr int kTcStagesX = 2 * kTcSlots;
-constexpr int kTcStagesA = 2 * kTcSlots;
+constexpr int kTcBK = 64;                 // k per shared-memory stage (one 128-byte swizzled row)
 constexpr int kTcThreads = 512;
-constexpr int kTcUnpackWarp0 = 4;
-constexpr int kTcPromoteWarp0 = 8;
-constexpr int kTcPromoteWarps = 8;
 constexpr uint32_t kTcTmemCols = 512;
-constexpr uint32_t kTmemT0 = 0, kTmemA = 256;
 constexpr int kTStride = 128;             // row stride (elements) of the low-rank [t_hi | t_lo] buffer
+// registers per thread of each warpgroup after setmaxnreg: producers/MMA, unpack, promotion x 2;
+// 128 * (48 + 96 + 2 * 184) = 512 threads * 128, the block's allocation at launch
+constexpr int kTcRegsWg0 = 48, kTcRegsWg1 = 96, kTcRegsPromote = 184, kTcRegsLaunch = 128;
+static_assert(kTcRegsWg0 + kTcRegsWg1 + 2 * kTcRegsPromote == 4 * kTcRegsLaunch, "register split");
 
-template <int BITS> struct TcStagesP { static constexpr int value = BITS <= 4 ? 8 : 5; };
-
-template <int BITS>
+template <int TT>
 struct TcLayout {
-    static constexpr int kSP = TcStagesP<BITS>::value;
-    static constexpr uint32_t kXBytes = kTcBT * kTcBK * 2;          // 16 KB
-    static constexpr uint32_t kPBytes = kTcBW * 16 * BITS;          // 128 rows x one group
+    static constexpr int kStages = TT == 256 ? 4 : 6;
+    static constexpr uint32_t kXBytes = TT * kTcBK * 2;             // 32 KB (TT = 256)
+    static constexpr uint32_t kABytes = kTcBW * kTcBK * 2;          // 16 KB
     static constexpr uint32_t kOffX = 0;
-    static constexpr uint32_t kOffP = kOffX + kTcStagesX * kXBytes;
-    static constexpr uint32_t kOffL = kOffP + kSP * kPBytes;       // low-rank L2 tile [rank][128] bf16
+    static constexpr uint32_t kOffA = kOffX + kStages * kXBytes;
+    static constexpr uint32_t kOffL = kOffA + kStages * kABytes;    // low-rank L2 tile [rank][128] bf16
     static constexpr uint32_t kLBytes = 64 * kTcBW * 2;
     static constexpr uint32_t kOffBar = kOffL + kLBytes;
-    static constexpr uint32_t kNumBars = 2 * kTcSlots + 2 * kSP + 2 + 2 + 2;
+    // full[S], empty[S], p_full[S], t_full[2], t_empty[2], l_full, l_empty, drain[2]
+    static constexpr uint32_t kNumBars = 3 * kStages + 8;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kBytes = kOffMisc + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;               // slack to align the base to 1024 B
 };
 
 struct TcParams {
+    const uint8_t *packed;    // N x K*b/8
     const float *scales;      // N x K/128
     const uint16_t *L2;       // rank x N bf16 or null
     const uint16_t *bias;     // N bf16 or null
     uint16_t *y;              // M x N bf16
     int64_t M, N, K;
+    int64_t row_bytes;        // K * b / 8
     int rank;
     int tiles_m, tiles_n;
     int l_tma;                // 1: the low-rank L2 tile of each weight tile arrives by TMA (l_map)
@@ -93,36 +94,69 @@ struct TcParams {
 // k stages (64 wide) of the low-rank unit: [t_hi | t_lo] has 2 * rank columns.
 __host__ __device__ constexpr int lowrank_stages(int rank) { return (2 * rank + kTcBK - 1) / kTcBK; }
 
-template <int BITS>
+template <int N> __device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N> __device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Named barrier 1 over the 128 unpack threads that also ORs a predicate across them: every
+// thread gets the same answer.
+__device__ __forceinline__ bool unpack_bar_any(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "barrier.cta.red.or.pred p, 1, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r) : "r"((uint32_t)pred) : "memory");
+    return r != 0;
+}
+
+// Byte offset of 16-byte chunk c (0..7) of row r in a tile of 128-byte rows stored in the
+// canonical K-major 128-byte-swizzle layout (8-row blocks of 1024 bytes, chunk index XOR
+// row mod 8) -- the layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B and the MMA reads.
+__device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) {
+    return (r >> 3) * 1024u + (r & 7u) * 128u + ((c ^ (r & 7u)) << 4);
+}
+
+template <int BITS, int TT>
 __global__ void __launch_bounds__(kTcThreads, 1)
-tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap p_map,
-                 const __grid_constant__ CUtensorMap t_map, const __grid_constant__ CUtensorMap l_map,
+tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap t_map,
+                 const __grid_constant__ CUtensorMap l_map, const __grid_constant__ CUtensorMap p_map,
                  const TcParams p) {
-    using L = TcLayout<BITS>;
-    constexpr int SP = L::kSP;
+    using L = TcLayout<TT>;
+    constexpr int S = L::kStages;
     constexpr int NWG = 4 * BITS + 1;
+    constexpr int kHalf = TT / 2;                 // promotion columns per warp
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
-    uint64_t *ready = bars, *consumed = ready + kTcSlots;
-    uint64_t *p_full = consumed + kTcSlots, *p_empty = p_full + SP;
-    uint64_t *t_full = p_empty + SP, *drain = t_full + 2;      // drain[2]: one per MMA thread
-    uint64_t *l_full = drain + 2, *l_empty = l_full + 1;        // low-rank L2 tile handoff
+    uint64_t *full = bars, *empty = full + S, *p_full = empty + S;
+    uint64_t *t_full = p_full + S, *t_empty = t_full + 2;
+    uint64_t *l_full = t_empty + 2, *l_empty = l_full + 1;
+    uint64_t *drain = l_empty + 1;                               // drain[2]: one per MMA thread
     const uint16_t *l_tile = reinterpret_cast<const uint16_t *>(smem + L::kOffL);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        // ready: x producer (1, plus transaction bytes) + 4 unpack warps + the promotion warps
-        for (int i = 0; i < kTcSlots; ++i) { mbar_init(&ready[i], 1 + 4 + kTcPromoteWarps); mbar_init(&consumed[i], 1); }
-        for (int i = 0; i < SP; ++i) { mbar_init(&p_full[i], 1); mbar_init(&p_empty[i], 4 * 32); }
-        for (int i = 0; i < 2; ++i) mbar_init(&t_full[i], 1);
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], 1 + 4);          // x producer (+ transaction bytes) + 4 unpack warps
+            mbar_init(&empty[i], 1);             // the commit of the MMAs that read the stage
+            mbar_init(&p_full[i], 1);            // packed group tile landed in this stage (TMA bytes)
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&t_full[i], 1);
+            mbar_init(&t_empty[i], 8);           // the 8 promotion warps
+        }
+        mbar_init(l_full, 1);
+        mbar_init(l_empty, 4);
         mbar_init(&drain[0], 1);
         mbar_init(&drain[1], 1);
-        mbar_init(l_full, 1);
-        mbar_init(l_empty, 4 * 32);
         *abort = 0;
         fence_barrier_init();
     }
@@ -136,165 +170,181 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
     const uint32_t tmem = *tmem_holder;
 
     const int G = (int)(p.K / 128);
+    const int nlr = p.rank > 0 ? lowrank_stages(p.rank) : 0;
     const int U = G + (p.rank > 0 ? 1 : 0);          // units per tile: groups (+ low-rank)
     const int tiles = p.tiles_m * p.tiles_n;
+    const int wg = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 7), 0);   // warp-uniform role
 
-    if (warp == 0 && lane == 0) {
-        // ---------------------------------------------------------- x / t producer
-        tma_prefetch_desc(&x_map);
-        tma_prefetch_desc(&t_map);
-        int armed[kTcSlots];
-        for (int i = 0; i < kTcSlots; ++i) armed[i] = -1;
-        uint32_t unit = 0;
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-            const int mt = tile % p.tiles_m;
-            for (int u = 0; u < U; ++u, ++unit) {
-                const uint32_t slot = unit % kTcSlots, ph = (unit / kTcSlots) & 1;
-                const int nst = (u < G) ? 2 : lowrank_stages(p.rank);
-                if (!mbar_wait(&consumed[slot], ph ^ 1, abort)) goto x_done;
-                mbar_arrive_expect_tx(&ready[slot], nst * L::kXBytes);
-                armed[slot] = (int)ph;
-                for (int st = 0; st < nst; ++st) {
-                    uint8_t *dst = smem + L::kOffX + (slot * 2 + st) * L::kXBytes;
-                    if (u < G) tma_load_2d(dst, &x_map, &ready[slot], (2 * u + st) * kTcBK, mt * kTcBT);
-                    else tma_load_2d(dst, &t_map, &ready[slot], st * kTcBK, mt * kTcBT);
-                }
-            }
-        }
-    x_done:
-        // wait (bounded) for the copies still in flight: a slot's phase cannot complete without
-        // them, so poll the transaction count through the phase of the last armed unit
-        for (int i = 0; i < kTcSlots; ++i) {
-            int local = 0;
-            if (armed[i] >= 0 && *abort) (void)mbar_wait(&ready[i], (uint32_t)armed[i], &local, 50ull * 1000ull * 1000ull);
-        }
-    } else if (warp == 2 && lane == 0) {
-        // ---------------------------------------------------------- packed-weight producer
-        tma_prefetch_desc(&p_map);
-        int armed[SP];
-        for (int i = 0; i < SP; ++i) armed[i] = -1;
-        if (p.l_tma) tma_prefetch_desc(&l_map);
-        uint32_t s = 0, ph = 0, lph = 0;
-        int l_armed = -1;
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-            const int nt = tile / p.tiles_m;
-            for (int g = 0; g < G; ++g) {
-                if (!mbar_wait(&p_empty[s], ph ^ 1, abort)) goto p_done;
-                mbar_arrive_expect_tx(&p_full[s], L::kPBytes);
-                armed[s] = (int)ph;
-                tma_load_2d(smem + L::kOffP + s * L::kPBytes, &p_map, &p_full[s], g * 16 * BITS, nt * kTcBW);
-                if (++s == SP) { s = 0; ph ^= 1; }
-            }
-            if (p.l_tma) {
-                // this tile's L2 columns, [rank][128 rows]; the tile's low-rank unit comes after all
-                // its groups, so the copy issued here lands long before it is read
-                if (!mbar_wait(l_empty, lph ^ 1, abort)) goto p_done;
-                mbar_arrive_expect_tx(l_full, (uint32_t)p.rank * kTcBW * 2);
-                l_armed = (int)lph;
-                tma_load_2d(smem + L::kOffL, &l_map, l_full, nt * kTcBW, 0);
-                lph ^= 1;
-            }
-        }
-    p_done:
-        for (int i = 0; i < SP; ++i) {
-            int local = 0;
-            if (armed[i] >= 0) (void)mbar_wait(&p_full[i], (uint32_t)armed[i], &local);
-        }
-        if (l_armed >= 0) {
-            int local = 0;
-            (void)mbar_wait(l_full, (uint32_t)l_armed, &local);
-        }
-    } else if ((warp == 1 || warp == 3) && lane == 0) {
-        // ---------------------------------------------------------- MMA issuers
-        // Two threads issue: warp 1 the even units (into T0), warp 3 the odd units (into T1).
-        // An MMA issue occupies the issuing thread for ~85 cycles and each unit also costs a
-        // barrier wait and two commits; a second issuer overlaps that with the other's MMAs.
-        const uint32_t mine = (warp == 1) ? 0u : 1u;
-        constexpr uint32_t idesc = umma_idesc_bf16(kTcBW, kTcBT);
-        uint32_t unit = 0;
-        const uint32_t x_base = smem_u32(smem + L::kOffX);
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-            for (int u = 0; u < U; ++u, ++unit) {
-                if ((unit & 1u) != mine) continue;
-                const uint32_t slot = unit % kTcSlots, ph = (unit / kTcSlots) & 1, tb = unit & 1;
-                if (!mbar_wait(&ready[slot], ph, abort)) goto m_done;
-                tc_fence_after();
-                const uint32_t d = tmem + kTmemT0 + tb * kTcBT;
-                const int nst = (u < G) ? 2 : lowrank_stages(p.rank);
-                for (int st = 0; st < nst; ++st) {
-                    const int nk = (u < G) ? kTcBK / 16 : min(kTcBK, 2 * p.rank - st * kTcBK) / 16;
-                    const uint32_t a = tmem + kTmemA + (slot * 2 + st) * (kTcBK / 2);
-                    const uint32_t b_base = x_base + (slot * 2 + st) * L::kXBytes;
-                    for (int k = 0; k < nk; ++k) {
-                        const uint64_t bd = umma_desc_sw128(b_base + k * 32, 1024);
-                        umma_bf16_ts(d, a + k * 8, bd, idesc, (st > 0 || k > 0) ? 1u : 0u);
+    if (wg == 0) {
+        regs_dec<kTcRegsWg0>();
+        if (warp == 0 && lane == 0) {
+            // ------------------------------------------------------ x / t producer
+            tma_prefetch_desc(&x_map);
+            tma_prefetch_desc(&t_map);
+            int armed[S];
+            for (int i = 0; i < S; ++i) armed[i] = -1;
+            uint32_t q = 0;
+            for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+                const int mt = tile / p.tiles_n;
+                for (int u = 0; u < U; ++u) {
+                    const int nst = (u < G) ? 2 : nlr;
+                    for (int st = 0; st < nst; ++st, ++q) {
+                        const uint32_t s = q % S, ph = (q / S) & 1;
+                        if (!mbar_wait(&empty[s], ph ^ 1, abort)) goto x_done;
+                        mbar_arrive_expect_tx(&full[s], L::kXBytes);
+                        armed[s] = (int)ph;
+                        uint8_t *dst = smem + L::kOffX + s * L::kXBytes;
+                        if (u < G) tma_load_2d(dst, &x_map, &full[s], (2 * u + st) * kTcBK, mt * TT);
+                        else tma_load_2d(dst, &t_map, &full[s], st * kTcBK, mt * TT);
                     }
                 }
-                umma_commit(&consumed[slot]);
-                umma_commit(&t_full[tb]);
             }
-        }
-    m_done:
-        {
-            // every MMA issued by this thread completes before TMEM is released
-            umma_commit(&drain[mine]);
-            int local = 0;
-            (void)mbar_wait(&drain[mine], 0, &local);
-        }
-    } else if (warp >= kTcUnpackWarp0 && warp < kTcPromoteWarp0) {
-        // ---------------------------------------------------------- unpack codes into TMEM
-        const int quarter = warp & 3;
-        const int row_local = quarter * 32 + lane;
-        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        uint32_t sp = 0, pp = 0, unit = 0, lph = 0;
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-            const int nt = tile / p.tiles_m;
-            const int64_t n = (int64_t)nt * kTcBW + row_local;
-            const bool row_ok = n < p.N;
-            for (int u = 0; u < U; ++u, ++unit) {
-                const uint32_t slot = unit % kTcSlots, ph = (unit / kTcSlots) & 1;
-                const uint32_t a_addr = tmem + lane_addr + kTmemA + slot * 2 * (kTcBK / 2);
-                if (u < G) {
-                    if (!warp_wait(&p_full[sp], pp, abort)) goto u_done;
-                    uint32_t w[NWG];
-                    {
-                        const uint4 *src = reinterpret_cast<const uint4 *>(smem + L::kOffP + sp * L::kPBytes +
-                                                                            row_local * 16 * BITS);
-#pragma unroll
-                        for (int i = 0; i < BITS; ++i) {
-                            const uint4 v = src[i];
-                            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-                        }
-                        w[4 * BITS] = 0;
+        x_done:
+            // wait (bounded) for the copies still in flight: a stage's phase cannot complete
+            // without them, so poll the transaction count through the last armed phase
+            for (int i = 0; i < S; ++i) {
+                int local = 0;
+                if (armed[i] >= 0 && *abort) (void)mbar_wait(&full[i], (uint32_t)armed[i], &local, 50ull * 1000ull * 1000ull);
+            }
+        } else if (warp == 2 && lane == 0) {
+            // ------------------------------------------------------ packed-code and L2 tile producer
+            // A group's packed tile (128 rows x 16*b bytes, <= 14 KB) lands in the code buffer of
+            // the unit's second stage, where the unpack warps read it before overwriting it with
+            // that stage's codes; the tile's L2 block goes to its own buffer once per tile.
+            tma_prefetch_desc(&p_map);
+            if (p.l_tma && p.rank > 0) tma_prefetch_desc(&l_map);
+            int armed[S];
+            for (int i = 0; i < S; ++i) armed[i] = -1;
+            int l_armed = -1;
+            uint32_t q = 0, lph = 0;
+            for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+                const int nt = tile % p.tiles_n;
+                for (int u = 0; u < G; ++u, q += 2) {
+                    const uint32_t s1 = (q + 1) % S, ph1 = ((q + 1) / S) & 1;
+                    if (!mbar_wait(&empty[s1], ph1 ^ 1, abort)) goto p_done;
+                    mbar_arrive_expect_tx(&p_full[s1], (uint32_t)kTcBW * 16u * BITS);
+                    armed[s1] = (int)ph1;
+                    tma_load_2d(smem + L::kOffA + s1 * L::kABytes, &p_map, &p_full[s1], u * 16 * BITS, nt * kTcBW);
+                }
+                if (p.rank > 0) {
+                    q += nlr;
+                    if (p.l_tma) {
+                        if (!mbar_wait(l_empty, lph ^ 1, abort)) goto p_done;
+                        mbar_arrive_expect_tx(l_full, (uint32_t)p.rank * kTcBW * 2);
+                        l_armed = (int)lph;
+                        tma_load_2d(smem + L::kOffL, &l_map, l_full, nt * kTcBW, 0);
+                        lph ^= 1;
                     }
-                    // Every consuming thread releases the stage itself (arrival count 128), after a
-                    // proxy fence: its loads are generic-proxy reads and the producer's next copy
-                    // is an async-proxy write, so the reads are ordered before the release across
-                    // proxies. (One lane's arrive after a warp sync let the next copy land while
-                    // other lanes' loads were in flight.)
-                    fence_proxy_async_smem();
-                    mbar_arrive(&p_empty[sp]);
-                    if (++sp == SP) { sp = 0; pp ^= 1; }
-                    uint32_t q0[32], q1[32];
-                    unpack_pairs<BITS, 0, 8>(w, q0);
-                    unpack_pairs<BITS, 8, 8>(w, q1);
-                    if (!warp_wait(&consumed[slot], ph ^ 1, abort)) goto u_done;
-                    tc_fence_after();        // order the stores after the MMAs that read this slot
-                    tmem_st_32x32b_x32(a_addr, q0);
-                    tmem_st_32x32b_x32(a_addr + kTcBK / 2, q1);
-                } else {
-                    // low-rank unit: A[n][k] = L2[k mod rank][n] for k < 2 rank (both halves of
-                    // [t_hi | t_lo] meet the same L2), zero beyond; from the shared-memory tile
-                    // when it came by TMA, else straight from global memory
-                    if (p.l_tma && !warp_wait(l_full, lph, abort)) goto u_done;
-                    if (!warp_wait(&consumed[slot], ph ^ 1, abort)) goto u_done;
+                }
+            }
+        p_done:
+            for (int i = 0; i < S; ++i) {
+                int local = 0;
+                if (armed[i] >= 0) (void)mbar_wait(&p_full[i], (uint32_t)armed[i], &local, 50ull * 1000ull * 1000ull);
+            }
+            if (l_armed >= 0) {
+                int local = 0;
+                (void)mbar_wait(l_full, (uint32_t)l_armed, &local, 50ull * 1000ull * 1000ull);
+            }
+        } else if ((warp == 1 || warp == 3) && lane == 0) {
+            // ------------------------------------------------------ MMA issuers
+            // Two threads issue: warp 1 the even units (into T0), warp 3 the odd units (into T1).
+            const uint32_t mine = (warp == 1) ? 0u : 1u;
+            constexpr uint32_t idesc = umma_idesc_bf16(kTcBW, TT);
+            const uint32_t x_base = smem_u32(smem + L::kOffX), a_base = smem_u32(smem + L::kOffA);
+            uint32_t q = 0, unit = 0;
+            for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+                for (int u = 0; u < U; ++u, ++unit) {
+                    const int nst = (u < G) ? 2 : nlr;
+                    if ((unit & 1u) != mine) { q += nst; continue; }
+                    const uint32_t tb = unit & 1;
+                    if (!mbar_wait(&t_empty[tb], ((unit >> 1) & 1) ^ 1, abort)) goto m_done;
                     tc_fence_after();
-                    const int nst = lowrank_stages(p.rank);
-                    for (int st = 0; st < nst; ++st) {
-                        uint32_t q[32];
+                    const uint32_t d = tmem + tb * TT;
+                    for (int st = 0; st < nst; ++st, ++q) {
+                        const uint32_t s = q % S, ph = (q / S) & 1;
+                        if (!mbar_wait(&full[s], ph, abort)) goto m_done;
+                        tc_fence_after();
+                        const int nk = (u < G) ? kTcBK / 16 : min(kTcBK, 2 * p.rank - st * kTcBK) / 16;
+                        const uint32_t xa = x_base + s * L::kXBytes, aa = a_base + s * L::kABytes;
+                        for (int k = 0; k < nk; ++k)
+                            umma_bf16(d, umma_desc_sw128(aa + k * 32, 1024), umma_desc_sw128(xa + k * 32, 1024), idesc,
+                                      (st > 0 || k > 0) ? 1u : 0u);
+                        umma_commit(&empty[s]);
+                    }
+                    umma_commit(&t_full[tb]);
+                }
+            }
+        m_done:
+            {
+                // every MMA issued by this thread completes before TMEM is released
+                umma_commit(&drain[mine]);
+                int local = 0;
+                (void)mbar_wait(&drain[mine], 0, &local);
+            }
+        }
+    } else if (wg == 1) {
+        regs_dec<kTcRegsWg1>();
+        // ---------------------------------------------------------- unpack codes into shared memory
+        const int row_local = threadIdx.x - 128;
+        const uint32_t a_base = smem_u32(smem + L::kOffA);
+        uint32_t q = 0, lph = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+            const int nt = tile % p.tiles_n;
+            const int64_t n = (int64_t)nt * kTcBW + row_local;
+            const bool row_ok = n < p.N;        // (rows past N arrive as zeros and are never stored)
+            for (int g = 0; g < G; ++g) {
+                const uint32_t s0 = q % S, ph0 = (q / S) & 1;
+                const uint32_t s1 = (q + 1) % S, ph1 = ((q + 1) / S) & 1;
+                q += 2;
+                // this row's packed group, from the tile the producer put in stage s1's code buffer
+                const bool got = warp_wait(&p_full[s1], ph1, abort);
+                uint32_t w[NWG];
+                w[4 * BITS] = 0;
+                if (got) {
+                    const uint8_t *src = smem + L::kOffA + s1 * L::kABytes + row_local * (16 * BITS);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const int k = st * kTcBK + 2 * i;
+                    for (int i = 0; i < BITS; ++i) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(src + 16 * i);
+                        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+                    }
+                }
+                const bool ready = got && warp_wait(&empty[s0], ph0 ^ 1, abort);
+                // every unpack thread has its row in registers before any code overwrites the
+                // tile; the barrier also votes, so that the four warps stop together when a wait
+                // gave up (a warp that left alone would strand the others at the next barrier)
+                if (unpack_bar_any(!ready)) goto u_done;
+                static_for<2>([&](auto st_) {
+                    constexpr int st = decltype(st_)::value;
+                    const uint32_t s = st == 0 ? s0 : s1;
+                    const uint32_t base = a_base + s * L::kABytes;
+                    static_for<8>([&](auto c_) {
+                        constexpr int c = decltype(c_)::value;
+                        uint32_t o[4];
+                        unpack_pairs<BITS, st * 8 + c, 1>(w, o);
+                        st_shared_v4(base + sw128_offset(row_local, c), o[0], o[1], o[2], o[3]);
+                    });
+                    // the MMA reads the tile through the async proxy
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full[s]);
+                });
+            }
+            if (p.rank > 0) {
+                // low-rank unit: A[n][k] = L2[k mod rank][n] for k < 2 rank (both halves of
+                // [t_hi | t_lo] meet the same L2), zero beyond; from the shared-memory tile when
+                // it came by TMA, else straight from global memory
+                if (p.l_tma && !warp_wait(l_full, lph, abort)) goto u_done;
+                for (int st = 0; st < nlr; ++st, ++q) {
+                    const uint32_t s = q % S, ph = (q / S) & 1;
+                    if (!warp_wait(&empty[s], ph ^ 1, abort)) goto u_done;
+                    const uint32_t base = a_base + s * L::kABytes;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t o[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int k = st * kTcBK + c * 8 + 2 * e;
                             uint32_t v = 0;
                             if (k < 2 * p.rank) {
                                 const int j = k < p.rank ? k : k - p.rank;
@@ -305,44 +355,43 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                                         ((uint32_t)__ldg(p.L2 + (int64_t)(j + 1) * p.N + n) << 16);
                                 }
                             }
-                            q[i] = v;
+                            o[e] = v;
                         }
-                        tmem_st_32x32b_x32(a_addr + st * (kTcBK / 2), q);
+                        st_shared_v4(base + sw128_offset(row_local, c), o[0], o[1], o[2], o[3]);
                     }
-                    if (p.l_tma) {
-                        // the tile is read: release it to the next tile's copy (per lane, after the
-                        // proxy fence, as for the packed stages)
-                        fence_proxy_async_smem();
-                        mbar_arrive(l_empty);
-                        lph ^= 1;
-                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full[s]);
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ready[slot]);
+                if (p.l_tma) {
+                    // the L2 tile is read: release it to the next tile's copy (generic reads before
+                    // the next async-proxy write)
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(l_empty);
+                    lph ^= 1;
+                }
             }
         }
     u_done:;
-    } else if (warp >= kTcPromoteWarp0) {
+    } else {
+        regs_inc<kTcRegsPromote>();
         // ---------------------------------------------------------- promotion + epilogue
         const int quarter = warp & 3;
-        const int colh = (warp - kTcPromoteWarp0) >> 2;            // which 64 token columns
+        const int colh = (warp - 8) >> 2;                          // which TT/2 token columns
         const int row_local = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         constexpr int kPre = 4;                                     // scale prefetch distance
-        // both T buffers start free: count this warp's release for units 0 and 1
-        if (lane == 0) { mbar_arrive(&ready[0]); mbar_arrive(&ready[1]); }
         uint32_t unit = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-            const int mt = tile % p.tiles_m, nt = tile / p.tiles_m;
+            const int mt = tile / p.tiles_n, nt = tile % p.tiles_n;
             const int64_t n = (int64_t)nt * kTcBW + row_local;
             const bool row_ok = n < p.N;
             const float *srow = p.scales + (row_ok ? n : 0) * (int64_t)G;
             float sq[kPre];
 #pragma unroll
             for (int i = 0; i < kPre; ++i) sq[i] = (row_ok && i < G) ? __ldg(srow + i) : 0.0f;
-            float R[64];
+            float R[kHalf];
             for (int u = 0; u < U; ++u, ++unit) {
                 float s = 1.0f;
                 if (u < G) {
@@ -354,17 +403,17 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                 const uint32_t tb = unit & 1, tph = (unit >> 1) & 1;
                 if (!warp_wait(&t_full[tb], tph, abort)) goto pr_done;
                 tc_fence_after();
-                const uint32_t t_addr = tmem + lane_addr + kTmemT0 + tb * kTcBT + colh * 64;
+                const uint32_t t_addr = tmem + lane_addr + tb * TT + colh * kHalf;
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
+                for (int hf = 0; hf < kHalf / 32; ++hf) {
                     uint32_t tv[32];
                     tmem_ld_32x32b_x32(t_addr + 32 * hf, tv);
                     tmem_wait_ld();
-                    if (hf == 1) {
-                        // both halves of T are in registers: hand the buffer back to the MMA
+                    if (hf == kHalf / 32 - 1) {
+                        // all of this warp's T columns are in registers: hand the buffer back
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&ready[(unit + 2) % kTcSlots]);
+                        if (lane == 0) mbar_arrive(&t_empty[tb]);
                     }
                     if (u == 0) {
 #pragma unroll
@@ -380,9 +429,9 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
             // ------------------------------------------------------ epilogue
             if (row_ok) {
                 const float bn = p.bias ? bf16_bits_to_f32(__ldg(p.bias + n)) : 0.0f;
-                const int64_t m0 = (int64_t)mt * kTcBT + colh * 64;
+                const int64_t m0 = (int64_t)mt * TT + colh * kHalf;
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
+                for (int j = 0; j < kHalf; ++j) {
                     if (m0 + j < p.M)
                         p.y[(m0 + j) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(R[j] + bn));
                 }

@@ -83,11 +83,42 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
     return d;
 }
 
+// abs_max of the group held by four consecutive lanes (32 bf16 weights, as 16 words, each):
+// a bf16x2 max-of-magnitudes tree, then two shuffles across the four lanes.
+__device__ __forceinline__ float group_abs_max(const uint32_t (&w)[16]) {
+    uint32_t m8[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m8[i] = bf16x2_maxabs(w[2 * i], w[2 * i + 1]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m8[i] = bf16x2_maxabs(m8[i], m8[i + 4]);
+    m8[0] = bf16x2_maxabs(m8[0], m8[2]);
+    m8[1] = bf16x2_maxabs(m8[1], m8[3]);
+    const uint32_t m2 = bf16x2_maxabs(m8[0], m8[1]) & 0x7FFF7FFFu;
+    uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    return __uint_as_float(m << 16);
+}
+
 __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
     uint4 v;
     asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
+}
+
+// step = RN(2 RN(abs_max * 1.01) / (2^b - 1)) of one group (see the header comment).
+template <int BITS>
+__device__ __forceinline__ float group_step(float abs_max) {
+    constexpr float kL = (float)((1 << BITS) - 1);
+    constexpr float kInvL = 1.0f / kL;                              // RN(1/L), folded by the compiler
+    const float two = __fmul_rn(2.0f, __fmul_rn(abs_max, 1.01f));
+    if (two >= 7.52316384526264e-37f && two <= 1.329227995784916e36f) {   // [2^-120, 2^120]
+        const float q0 = __fmul_rn(two, kInvL);
+        const float r = __fmaf_rn(-q0, kL, two);
+        return __fmaf_rn(r, kInvL, q0);
+    }
+    return __fdiv_rn(two, kL);
 }
 
 template <int BITS>
@@ -102,13 +133,10 @@ template <int BITS, bool DIRECT>
 __device__ __forceinline__ void pack_block(const uint16_t *__restrict__ W, int64_t n_groups,
                                            uint8_t *__restrict__ packed, float *__restrict__ scales,
                                            int64_t g0, uint32_t *stage_w, int lane) {
-    constexpr int kLevels = (1 << BITS) - 1;
     constexpr int kOff = 1 << (BITS - 1);
     constexpr int kGroupBytes = 16 * BITS;
     constexpr int U = kPackUnroll;
     constexpr int GW = kPackGroupsPerWarp;
-    constexpr float kL = (float)kLevels;
-    constexpr float kInvL = 1.0f / (float)kLevels;                  // RN(1/L), folded by the compiler
     constexpr float kMagicA = 12582912.0f;                          // 1.5 * 2^23
     constexpr float kMagicB = 8388608.0f + (float)(kOff * ((1 << BITS) + 1));
     constexpr float kPow = (float)(1 << BITS);
@@ -129,29 +157,8 @@ __device__ __forceinline__ void pack_block(const uint16_t *__restrict__ W, int64
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         const int64_t g = g0 + 8 * u + gi;
-        // ---- abs_max of the group (bf16 magnitudes; the max tree keeps only |.|)
-        uint32_t m8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = bf16x2_maxabs(w[u][2 * i], w[u][2 * i + 1]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) m8[i] = bf16x2_maxabs(m8[i], m8[i + 4]);
-        m8[0] = bf16x2_maxabs(m8[0], m8[2]);
-        m8[1] = bf16x2_maxabs(m8[1], m8[3]);
-        const uint32_t m2 = bf16x2_maxabs(m8[0], m8[1]) & 0x7FFF7FFFu;
-        uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        const float abs_max = __uint_as_float(m << 16);
-        // ---- step = RN(2 s / L), s = RN(abs_max * 1.01)
-        const float two = __fmul_rn(2.0f, __fmul_rn(abs_max, 1.01f));
-        float step;
-        if (two >= 7.52316384526264e-37f && two <= 1.329227995784916e36f) {   // [2^-120, 2^120]
-            const float q0 = __fmul_rn(two, kInvL);
-            const float r = __fmaf_rn(-q0, kL, two);
-            step = __fmaf_rn(r, kInvL, q0);
-        } else {
-            step = __fdiv_rn(two, kL);
-        }
+        // ---- abs_max of the group (bf16 magnitudes; the max tree keeps only |.|), then the step
+        const float step = group_step<BITS>(group_abs_max(w[u]));
         float inv = (step == 0.0f) ? 0.0f : __frcp_rn(step);
         bool near = !(inv <= 3.402823466e38f);           // 1/step overflowed: divide always
         if (near) inv = 0.0f;

@@ -18,8 +18,11 @@
 
 #include "common.cuh"
 #include "pack.cuh"
+#include "error.cuh"
+#include "dequant.cuh"
 #include "smallm.cuh"
 #include "gemm_tc.cuh"
+#include "pd_search.h"
 
 namespace {
 
@@ -138,65 +141,56 @@ wq_status launch_pack_many(const wq_pack_job *jobs, int n_jobs, int sm_count, cu
     return WQ_OK;
 }
 
+// ------------------------------------------------------------------ error table
+// The jobs' outputs are zeroed, then quant_error_many_kernel runs over up to kErrMaxSegs
+// tensors per launch.
+wq_status launch_error_many(const wq_error_job *jobs, int n_jobs, int sm_count, cudaStream_t st) {
+    wq::ErrSegments segs;
+    int i = 0;
+    while (i < n_jobs) {
+        segs.n = 0;
+        segs.vbegin[0] = 0;
+        for (; i < n_jobs && segs.n < wq::kErrMaxSegs; ++i) {
+            const wq_error_job &j = jobs[i];
+            const int k = segs.n++;
+            const int64_t n_groups = j.N * (j.K / 128);
+            segs.n_groups[k] = n_groups;
+            segs.W[k] = static_cast<const uint16_t *>(j.W);
+            segs.out[k] = j.out;
+            segs.vbegin[k + 1] = segs.vbegin[k] + (n_groups + 7) / 8 * 8;
+        }
+        wq::zero_error_outputs_kernel<<<1, wq::kErrMaxSegs * wq::kErrOut, 0, st>>>(segs);
+        wq_status s = check_launch("zero_error_outputs_kernel");
+        if (s != WQ_OK) return s;
+        const int64_t per_block = 8 * (wq::kErrThreads / 32);
+        const int64_t want = (segs.vbegin[segs.n] + per_block - 1) / per_block;
+        if (want > 0) {
+            const int grid = (int)std::min<int64_t>(want, (int64_t)sm_count * 12);
+            wq::quant_error_many_kernel<<<grid, wq::kErrThreads, 0, st>>>(segs);
+            if ((s = check_launch("quant_error_many_kernel")) != WQ_OK) return s;
+        }
+    }
+    return WQ_OK;
+}
+
 // ------------------------------------------------------------------ small-M path
 constexpr uint32_t kSmemMax = 227 * 1024;        // dynamic shared memory per CTA on sm_100
 
 uint32_t align_u32(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-// Stage and shared-memory layout of smallm_kernel for `rows` weight rows per stage and a
-// CTA range of `gcta` groups (`even`: every CTA of the launch has exactly gcta groups).
-// Chunk width gc: the largest candidate that keeps a ring of at least three stages (two at
-// one group per chunk); with an even split the candidates are the divisors of gcta, so no
-// chunk is short. gc * bits <= 64 keeps a weight box row within 256 32-bit words.
-template <int TOK>
-bool small_layout(int bits, int rows, int gcta, bool even, bool scale_tma, int sbox, wq::SmallMArgs &a,
-                  uint32_t *total) {
-    using T = wq::SmTok<TOK>;
-    const uint32_t tree = 4u * T::kNR * 32u * 4u;
-    const uint32_t part = align_u32((uint32_t)TOK * T::kPStride * 4u, 128);
-    const uint32_t bars = (2u * wq::kSmMaxStages + 4u) * 8u + 16u;
-    const uint32_t sres = scale_tma ? align_u32((uint32_t)rows * (uint32_t)sbox * 4u, 128) : 0u;
-    if (tree + part + bars + sres >= kSmemMax) return false;
-    const uint32_t budget = kSmemMax - tree - part - bars - sres;
-    for (int gc = std::min(gcta, 64 / bits); gc >= 1; --gc) {
-        if (even ? (gcta % gc != 0) : ((gc & (gc - 1)) != 0 || gc > 8)) continue;
-        const uint32_t w_bytes = align_u32((uint32_t)rows * (uint32_t)gc * 16u * (uint32_t)bits, 128);
-        const uint32_t x_bytes = align_u32((uint32_t)TOK * (uint32_t)gc * 256u, 128);
-        const uint32_t s_bytes = scale_tma ? 0u : align_u32((uint32_t)gc * (uint32_t)rows * 4u, 128);
-        const uint32_t stage = w_bytes + x_bytes + s_bytes;
-        const uint32_t stages = std::min<uint32_t>(wq::kSmMaxStages, budget / stage);
-        if (stages < 3 && !(gc == 1 && stages >= 2)) continue;
-        a.gc = gc;
-        a.stages = (int)stages;
-        a.srows = rows;
-        a.stage_bytes = stage;
-        a.off_x = w_bytes;
-        a.off_s = w_bytes + x_bytes;
-        a.scale_tma = scale_tma ? 1 : 0;
-        a.sbox = sbox;
-        a.off_sres = stages * stage;
-        a.off_tree = a.off_sres + sres;
-        a.off_part = a.off_tree + tree;
-        a.off_bar = a.off_part + part;
-        *total = a.off_bar + bars;
-        return true;
-    }
-    return false;
-}
-
 // Clusters of S CTAs that fit at once (one CTA per SM, the most shared memory), cached.
 template <int BITS, int TOK>
 int small_max_clusters(int dev, int S, int sm_count) {
     // computed once per device and cluster size; two threads racing here compute the same value
-    static std::atomic<int> cache[kMaxDevices][3] = {};
-    const int si = S == 1 ? 0 : (S == 2 ? 1 : 2);
+    static std::atomic<int> cache[kMaxDevices][4] = {};
+    const int si = S == 1 ? 0 : (S == 2 ? 1 : (S == 4 ? 2 : 3));
     const int cached = cache[dev][si].load(std::memory_order_relaxed);
     if (cached != 0) return cached;
     int n = sm_count / S;
     if (S > 1) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(S * (sm_count / S)));
-        cfg.blockDim = dim3(wq::kSmThreads);
+        cfg.blockDim = dim3(wq::SmCfg<TOK>::kThreads);
         cfg.dynamicSmemBytes = kSmemMax;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -215,15 +209,50 @@ int small_max_clusters(int dev, int S, int sm_count) {
     return v;
 }
 
-wq_status get_encoder();
-wq_status make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
-                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
-wq_status make_map_3d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, const uint64_t (&dims)[3],
-                      const uint64_t (&strides)[2], const uint32_t (&box)[3]);
+// Work split and shared-memory layout of smallm_kernel for a cluster size S: C clusters own
+// ~U/C units each, a CTA ~G/S groups. Inside the CTA, blocks of RB units go to the W warps
+// (GW warps per block, each a share of the groups, when there are fewer blocks than warps);
+// each warp streams its items through D ring slots. Returns the busiest warp's item count,
+// or -1 when nothing fits in shared memory.
+template <int BITS, int TOK>
+int64_t small_plan(int64_t U, int G, int S, int C, wq::SmallMArgs &a, uint32_t *smem_total) {
+    constexpr int W = wq::SmCfg<TOK>::kWarps;
+    const int64_t uc = (U + C - 1) / C;
+    const int gc = (G + S - 1) / S;
+    const uint32_t x_stride = (uint32_t)gc * 256u + 64u;
+    const uint32_t x_bytes = align_u32((uint32_t)TOK * x_stride, 128);
+    const uint32_t slot = 16u * 16u * BITS + 64u;
+    int64_t best = -1;
+    for (int rb = wq::kSmMaxRB; rb >= 1; --rb) {
+        const int64_t nb = (uc + rb - 1) / rb;
+        const int gw = nb >= W ? 1 : (int)(W / nb);
+        const int64_t items = nb >= W ? ((nb + W - 1) / W) * rb * gc : (int64_t)rb * ((gc + gw - 1) / gw);
+        const uint32_t part = align_u32((uint32_t)gw * TOK * (uint32_t)(uc * 16) * 4u, 128);
+        for (int d = wq::kSmMaxD; d >= 2; --d) {
+            const uint32_t total = x_bytes + (uint32_t)W * d * slot + part;
+            if (total > kSmemMax) continue;
+            // fewer items per warp first; then a deeper ring, then more x reuse (larger blocks)
+            const int64_t cost = items * 8 + (d >= 4 ? 0 : 4 - d);
+            if (best < 0 || cost < best) {
+                best = cost;
+                a.RB = rb;
+                a.GW = gw;
+                a.D = d;
+                a.rows_max = (int)(uc * 16);
+                a.x_stride = x_stride;
+                a.slot_bytes = slot;
+                a.off_ring = x_bytes;
+                a.off_part = x_bytes + (uint32_t)W * d * slot;
+                *smem_total = total;
+            }
+            break;
+        }
+    }
+    return best;
+}
 
 template <int BITS, int TOK>
-wq_status launch_smallm_tok(wq::SmallMArgs a, const uint8_t *packed, int dev, int sm_count, cudaStream_t st) {
-    using T = wq::SmTok<TOK>;
+wq_status launch_smallm_tok(wq::SmallMArgs a, int dev, int sm_count, cudaStream_t st) {
     static std::atomic<int> attr_done[kMaxDevices] = {};
     cudaError_t e = setup_once(attr_done, dev, [] {
         return cudaFuncSetAttribute(wq::smallm_kernel<BITS, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -232,83 +261,49 @@ wq_status launch_smallm_tok(wq::SmallMArgs a, const uint8_t *packed, int dev, in
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smallm)");
     const int64_t U = (a.N + 15) / 16;
     const int G = (int)(a.K / 128);
-    // cluster size S (K split) and cluster count C: the fewest items on the busiest CTA,
-    // items = (16-row units per cluster) x (groups per CTA); ties go to the smaller S
-    int bestS = 1, bestC = 1;
+    // cluster size S (K split) and cluster count C: the fewest items on the busiest warp;
+    // ties go to the smaller S
     int64_t best = -1;
-    for (int S = 1; S <= 4; S *= 2) {
+    wq::SmallMArgs chosen = a;
+    uint32_t smem = 0;
+    for (int S = 1; S <= 8; S *= 2) {
         if (S > G) break;
         const int mc = small_max_clusters<BITS, TOK>(dev, S, sm_count);
         if (mc <= 0) continue;
         const int C = (int)std::min<int64_t>(mc, U);
-        const int64_t cost = ((U + C - 1) / C) * ((G + S - 1) / S);
-        if (best < 0 || cost < best) { best = cost; bestS = S; bestC = C; }
+        wq::SmallMArgs t = a;
+        uint32_t total = 0;
+        const int64_t cost = small_plan<BITS, TOK>(U, G, S, C, t, &total);
+        if (cost < 0) continue;
+        if (best < 0 || cost < best) {
+            best = cost;
+            t.S = S;
+            t.n_clusters = C;
+            chosen = t;
+            smem = total;
+        }
     }
-    a.S = bestS;
-    a.n_clusters = bestC;
-    const int rows = (int)std::min<int64_t>(T::kRP, (U + bestC - 1) / bestC) * 16;
-    const int gcta = (G + bestS - 1) / bestS;
-    const bool even = (G % bestS) == 0;
-    // resident steps by TMA: rows of G fp32 must be 16-byte multiples; the box covers the
-    // CTA's groups from the 4-aligned group below its first one
-    const int sbox = (gcta + 3 + 3) / 4 * 4;
-    bool scale_tma = (G % 4 == 0) && sbox <= 256 && (uint64_t)rows * sbox * 4 <= 48 * 1024;
-    uint32_t smem = 0;
-    if (!small_layout<TOK>(BITS, rows, gcta, even, scale_tma, sbox, a, &smem)) {
-        scale_tma = false;
-        if (!small_layout<TOK>(BITS, rows, gcta, even, false, sbox, a, &smem))
-            return fail(WQ_ERR_INVALID_ARG, "no shared-memory layout for the small-M kernel");
-    }
-    // TMA maps: packed as [N][K*b/32] 32-bit words (boxes of gc groups x 64/32/16 rows) and,
-    // for short chunks, as {16b bytes, G, N} one group at a time; x as {128 k, G, M};
-    // steps as [N][G] fp32
-    const uint64_t G64 = (uint64_t)G, kGB = 16u * BITS, row_bytes = (uint64_t)a.K * BITS / 8;
-    CUtensorMap pm64, pm32, pm16, pm_tail, xm_full, xm_tail, sm_map;
-    wq_status s;
-    const uint64_t pdims[3] = {kGB, G64, (uint64_t)a.N};
-    const uint64_t pstr[2] = {kGB, row_bytes};
-    const uint64_t xdims[3] = {128, G64, (uint64_t)a.M};
-    const uint64_t xstr[2] = {256, (uint64_t)a.K * 2};
-    const uint32_t pbox_t[3] = {(uint32_t)kGB, 1, 16};
-    const uint32_t xbox_f[3] = {128, (uint32_t)a.gc, (uint32_t)TOK}, xbox_t[3] = {128, 1, (uint32_t)TOK};
-    const uint32_t wbox = (uint32_t)a.gc * 4u * BITS;
-    if ((s = make_map_2d(&pm64, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, row_bytes / 4, (uint64_t)a.N, row_bytes, wbox, 64,
-                         CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK ||
-        (s = make_map_2d(&pm32, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, row_bytes / 4, (uint64_t)a.N, row_bytes, wbox, 32,
-                         CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK ||
-        (s = make_map_2d(&pm16, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, row_bytes / 4, (uint64_t)a.N, row_bytes, wbox, 16,
-                         CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK ||
-        (s = make_map_3d(&pm_tail, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, pdims, pstr, pbox_t)) != WQ_OK ||
-        (s = make_map_3d(&xm_full, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, xdims, xstr, xbox_f)) != WQ_OK ||
-        (s = make_map_3d(&xm_tail, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, xdims, xstr, xbox_t)) != WQ_OK)
-        return s;
-    if (scale_tma) {
-        if ((s = make_map_2d(&sm_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.scales, G64, (uint64_t)a.N, G64 * 4,
-                             (uint32_t)sbox, 16, CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK)
-            return s;
-    } else {
-        sm_map = pm16;   // not read by the kernel
-    }
+    if (best < 0) return fail(WQ_ERR_INVALID_ARG, "no shared-memory layout for the small-M kernel");
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(bestC * bestS));
-    cfg.blockDim = dim3(wq::kSmThreads);
+    cfg.gridDim = dim3((unsigned)(chosen.n_clusters * chosen.S));
+    cfg.blockDim = dim3(wq::SmCfg<TOK>::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)bestS;
+    attr[0].val.clusterDim.x = (unsigned)chosen.S;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = bestS > 1 ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, wq::smallm_kernel<BITS, TOK>, pm64, pm32, pm16, pm_tail, xm_full, xm_tail, sm_map, a);
+    cfg.numAttrs = chosen.S > 1 ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, wq::smallm_kernel<BITS, TOK>, chosen);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(smallm_kernel)");
     return check_launch("smallm_kernel");
 }
 
 // Up to 16 tokens per launch; more tokens take several launches.
 template <int BITS>
-wq_status launch_smallm(const wq::SmallMArgs &base, const uint8_t *packed, int dev, int sm_count, cudaStream_t st) {
+wq_status launch_smallm(const wq::SmallMArgs &base, int dev, int sm_count, cudaStream_t st) {
     for (int64_t m0 = 0; m0 < base.M; m0 += wq::kSmMaxTok) {
         wq::SmallMArgs a = base;
         a.M = std::min<int64_t>(wq::kSmMaxTok, base.M - m0);
@@ -316,8 +311,8 @@ wq_status launch_smallm(const wq::SmallMArgs &base, const uint8_t *packed, int d
         a.y = base.y + m0 * base.N;
         if (base.t) a.t = base.t + m0 * wq::kTStrideSm;
         wq_status s;
-        if (a.M <= 8) s = launch_smallm_tok<BITS, 8>(a, packed, dev, sm_count, st);
-        else s = launch_smallm_tok<BITS, 16>(a, packed, dev, sm_count, st);
+        if (a.M <= 8) s = launch_smallm_tok<BITS, 8>(a, dev, sm_count, st);
+        else s = launch_smallm_tok<BITS, 16>(a, dev, sm_count, st);
         if (s != WQ_OK) return s;
     }
     return WQ_OK;
@@ -376,46 +371,47 @@ wq_status make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base
     return WQ_OK;
 }
 
-wq_status make_map_3d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, const uint64_t (&dims)[3],
-                      const uint64_t (&strides)[2], const uint32_t (&box)[3]) {
-    wq_status s = get_encoder();
-    if (s != WQ_OK) return s;
-    const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
-    const cuuint64_t st[2] = {strides[0], strides[1]};
-    const cuuint32_t b[3] = {box[0], box[1], box[2]};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = g_encode(map, dt, 3, const_cast<void *>(base), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(WQ_ERR_CUDA, "cuTensorMapEncodeTiled (3d) failed (%d)", (int)r);
-    return WQ_OK;
-}
-
-template <int BITS>
-wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &pm, const CUtensorMap &tm,
-                    const CUtensorMap &lm, int l_tma, int sm_count, cudaStream_t st) {
-    using L = wq::TcLayout<BITS>;
+template <int BITS, int TT>
+wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &tm, const CUtensorMap &lm,
+                    const CUtensorMap &pm, int l_tma, int sm_count, cudaStream_t st) {
+    using L = wq::TcLayout<TT>;
     static std::atomic<int> attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     const cudaError_t e = setup_once(attr_done, dev, [] {
-        return cudaFuncSetAttribute(wq::tc_linear_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        // The warpgroups re-split their registers with setmaxnreg, a split that adds up to
+        // exactly 128 registers per thread at launch: a kernel built with any other count
+        // would wait forever in setmaxnreg.inc, so it is never launched.
+        cudaFuncAttributes fa;
+        cudaError_t r = cudaFuncGetAttributes(&fa, wq::tc_linear_kernel<BITS, TT>);
+        if (r != cudaSuccess) return r;
+        if (fa.numRegs != wq::kTcRegsLaunch || fa.maxThreadsPerBlock < wq::kTcThreads) return cudaErrorInvalidKernelImage;
+        return cudaFuncSetAttribute(wq::tc_linear_kernel<BITS, TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)L::kAlloc);
     });
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc_linear_kernel)");
+    if (e != cudaSuccess) return cuda_fail(e, "tc_linear_kernel set-up (register count / shared memory)");
     wq::TcParams p{};
+    p.packed = a.packed;
     p.scales = a.scales;
     p.L2 = static_cast<const uint16_t *>(a.L2);
     p.bias = static_cast<const uint16_t *>(a.bias);
     p.y = static_cast<uint16_t *>(a.y);
     p.M = a.M; p.N = a.N; p.K = a.K; p.rank = a.rank;
-    p.tiles_m = (int)((a.M + wq::kTcBT - 1) / wq::kTcBT);
+    p.row_bytes = a.K * BITS / 8;
+    p.tiles_m = (int)((a.M + TT - 1) / TT);
     p.tiles_n = (int)((a.N + wq::kTcBW - 1) / wq::kTcBW);
     p.l_tma = l_tma;
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = std::min(tiles, sm_count);
-    wq::tc_linear_kernel<BITS><<<grid, wq::kTcThreads, L::kAlloc, st>>>(xm, pm, tm, lm, p);
+    wq::tc_linear_kernel<BITS, TT><<<grid, wq::kTcThreads, L::kAlloc, st>>>(xm, tm, lm, pm, p);
     return check_launch("tc_linear_kernel");
+}
+
+template <int BITS>
+wq_status launch_tc_tt(const TcArgs &a, int tt, const CUtensorMap &xm, const CUtensorMap &tm, const CUtensorMap &lm,
+                       const CUtensorMap &pm, int l_tma, int sm_count, cudaStream_t st) {
+    return tt == 256 ? launch_tc<BITS, 256>(a, xm, tm, lm, pm, l_tma, sm_count, st)
+                     : launch_tc<BITS, 128>(a, xm, tm, lm, pm, l_tma, sm_count, st);
 }
 
 template <int R>
@@ -453,16 +449,23 @@ wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_
     return check_launch("lowrank_prepass_kernel");
 }
 
+// Tokens per tensor-core tile: 256 (one MMA covers 128 weight rows x 256 tokens, which hides
+// the per-group hand-off of the partial products), 128 when there are few tokens.
+int tc_tile_tokens(int64_t M) { return M > 128 ? 256 : 128; }
+
 wq_status tc_linear(const TcArgs &a, int sm_count, cudaStream_t st) {
     wq_status s = get_encoder();
     if (s != WQ_OK) return s;
     if (a.M > (int64_t)INT32_MAX || a.N > (int64_t)INT32_MAX || a.K > (int64_t)INT32_MAX)
         return fail(WQ_ERR_INVALID_ARG, "dimension above 2^31 on the tensor-core path");
-    CUtensorMap xm, pm, tm, lm;
+    const int tt = tc_tile_tokens(a.M);
+    CUtensorMap xm, tm, lm;
     int l_tma = 0;
     if ((s = make_map_2d(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)a.K, (uint64_t)a.M,
-                         (uint64_t)a.K * 2, wq::kTcBK, wq::kTcBT, CU_TENSOR_MAP_SWIZZLE_128B)) != WQ_OK)
+                         (uint64_t)a.K * 2, wq::kTcBK, (uint32_t)tt, CU_TENSOR_MAP_SWIZZLE_128B)) != WQ_OK)
         return s;
+    // packed codes as [N][K*b/8] bytes: one group of 128 rows (16*b bytes each) per copy
+    CUtensorMap pm;
     const uint64_t row_bytes = (uint64_t)a.K * a.bits / 8;
     if ((s = make_map_2d(&pm, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.packed, row_bytes, (uint64_t)a.N, row_bytes,
                          16u * a.bits, wq::kTcBW, CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK)
@@ -478,7 +481,7 @@ wq_status tc_linear(const TcArgs &a, int sm_count, cudaStream_t st) {
         }
         if (s != WQ_OK) return s;
         if ((s = make_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, t, (uint64_t)wq::kTStride, (uint64_t)a.M,
-                             (uint64_t)wq::kTStride * 2, wq::kTcBK, wq::kTcBT, CU_TENSOR_MAP_SWIZZLE_128B)) != WQ_OK)
+                             (uint64_t)wq::kTStride * 2, wq::kTcBK, (uint32_t)tt, CU_TENSOR_MAP_SWIZZLE_128B)) != WQ_OK)
             return s;
         // L2 (rank x N) by TMA when its rows are 16-byte multiples: a [rank][128] tile per weight tile
         if (a.N % 8 == 0) {
@@ -490,11 +493,11 @@ wq_status tc_linear(const TcArgs &a, int sm_count, cudaStream_t st) {
     }
     if (!l_tma) lm = xm;   // not read by the kernel
     switch (a.bits) {
-        case 3: return launch_tc<3>(a, xm, pm, tm, lm, l_tma, sm_count, st);
-        case 4: return launch_tc<4>(a, xm, pm, tm, lm, l_tma, sm_count, st);
-        case 5: return launch_tc<5>(a, xm, pm, tm, lm, l_tma, sm_count, st);
-        case 6: return launch_tc<6>(a, xm, pm, tm, lm, l_tma, sm_count, st);
-        default: return launch_tc<7>(a, xm, pm, tm, lm, l_tma, sm_count, st);
+        case 3: return launch_tc_tt<3>(a, tt, xm, tm, lm, pm, l_tma, sm_count, st);
+        case 4: return launch_tc_tt<4>(a, tt, xm, tm, lm, pm, l_tma, sm_count, st);
+        case 5: return launch_tc_tt<5>(a, tt, xm, tm, lm, pm, l_tma, sm_count, st);
+        case 6: return launch_tc_tt<6>(a, tt, xm, tm, lm, pm, l_tma, sm_count, st);
+        default: return launch_tc_tt<7>(a, tt, xm, tm, lm, pm, l_tma, sm_count, st);
     }
 }
 
@@ -582,6 +585,36 @@ wq_status wq_quantize_pack(const void *W, int64_t N, int64_t K, int bits, int gr
     }
 }
 
+wq_status wq_dequantize(const uint8_t *packed, const float *scales, int64_t N, int64_t K, int bits, int group,
+                        void *W_hat, wq_stream_t stream) {
+    g_last_error[0] = 0;
+    if (bits < 3 || bits > 7) return fail(WQ_ERR_UNSUPPORTED_BITS, "bits=%d", bits);
+    if (group != 128) return fail(WQ_ERR_UNSUPPORTED_GROUP, "group=%d", group);
+    if (N < 0 || K < 0) return fail(WQ_ERR_INVALID_ARG, "negative size N=%lld K=%lld", (long long)N, (long long)K);
+    if (K % 128 != 0) return fail(WQ_ERR_INVALID_ARG, "K=%lld is not a multiple of 128", (long long)K);
+    if (N == 0 || K == 0) return WQ_OK;
+    if (!packed || !scales || !W_hat) return fail(WQ_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (!aligned16(packed) || !aligned16(scales) || !aligned16(W_hat))
+        return fail(WQ_ERR_MISALIGNED, "packed/scales/W_hat must be 16-byte aligned");
+    int dev;
+    const DeviceInfo *info;
+    wq_status s = current_device(&dev, &info);
+    if (s != WQ_OK) return s;
+    const int64_t n_groups = N * (K / 128);
+    const int64_t per_block = 8 * (wq::kDeqThreads / 32);
+    const int grid = (int)std::min<int64_t>((n_groups + per_block - 1) / per_block, (int64_t)info->sm_count * 8);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint16_t *out = static_cast<uint16_t *>(W_hat);
+    switch (bits) {
+        case 3: wq::dequantize_kernel<3><<<grid, wq::kDeqThreads, 0, st>>>(packed, scales, n_groups, out); break;
+        case 4: wq::dequantize_kernel<4><<<grid, wq::kDeqThreads, 0, st>>>(packed, scales, n_groups, out); break;
+        case 5: wq::dequantize_kernel<5><<<grid, wq::kDeqThreads, 0, st>>>(packed, scales, n_groups, out); break;
+        case 6: wq::dequantize_kernel<6><<<grid, wq::kDeqThreads, 0, st>>>(packed, scales, n_groups, out); break;
+        default: wq::dequantize_kernel<7><<<grid, wq::kDeqThreads, 0, st>>>(packed, scales, n_groups, out); break;
+    }
+    return check_launch("dequantize_kernel");
+}
+
 wq_status wq_quantize_pack_many(const wq_pack_job *jobs, int n_jobs, int group, wq_stream_t stream) {
     g_last_error[0] = 0;
     if (group != 128) return fail(WQ_ERR_UNSUPPORTED_GROUP, "group=%d", group);
@@ -612,6 +645,60 @@ wq_status wq_quantize_pack_many(const wq_pack_job *jobs, int n_jobs, int group, 
     if ((s = launch_pack_many<5>(jobs, n_jobs, info->sm_count, st)) != WQ_OK) return s;
     if ((s = launch_pack_many<6>(jobs, n_jobs, info->sm_count, st)) != WQ_OK) return s;
     return launch_pack_many<7>(jobs, n_jobs, info->sm_count, st);
+}
+
+wq_status wq_quant_error_many(const wq_error_job *jobs, int n_jobs, int group, wq_stream_t stream) {
+    g_last_error[0] = 0;
+    if (group != 128) return fail(WQ_ERR_UNSUPPORTED_GROUP, "group=%d", group);
+    if (n_jobs < 0) return fail(WQ_ERR_INVALID_ARG, "n_jobs=%d", n_jobs);
+    if (n_jobs == 0) return WQ_OK;
+    if (!jobs) return fail(WQ_ERR_INVALID_ARG, "NULL job array");
+    for (int i = 0; i < n_jobs; ++i) {
+        const wq_error_job &j = jobs[i];
+        if (j.N < 0 || j.K < 0)
+            return fail(WQ_ERR_INVALID_ARG, "job %d: negative size N=%lld K=%lld", i, (long long)j.N, (long long)j.K);
+        if (j.K % 128 != 0) return fail(WQ_ERR_INVALID_ARG, "job %d: K=%lld is not a multiple of 128", i, (long long)j.K);
+        if (!j.out || (j.N > 0 && j.K > 0 && !j.W)) return fail(WQ_ERR_INVALID_ARG, "job %d: NULL pointer", i);
+        if ((reinterpret_cast<uintptr_t>(j.out) & 7u) != 0 || (j.W && !aligned16(j.W)))
+            return fail(WQ_ERR_MISALIGNED, "job %d: W must be 16-byte and out 8-byte aligned", i);
+    }
+    int dev;
+    const DeviceInfo *info;
+    wq_status s = current_device(&dev, &info);
+    if (s != WQ_OK) return s;
+    return launch_error_many(jobs, n_jobs, info->sm_count, reinterpret_cast<cudaStream_t>(stream));
+}
+
+wq_status wq_quant_error(const void *W, int64_t N, int64_t K, int group, double *out, wq_stream_t stream) {
+    const wq_error_job job{W, N, K, out};
+    return wq_quant_error_many(&job, 1, group, stream);
+}
+
+wq_status wq_pd_search(const double *mse_table, const int64_t *n_params, int n_tensors, const int *bits, int n_bits,
+                       double target_bpw, int n_iters, int n_restarts, const double *t_init, int *bits_out,
+                       double *result) {
+    g_last_error[0] = 0;
+    if (n_tensors <= 0 || n_bits <= 0 || n_iters < 0 || n_restarts <= 0)
+        return fail(WQ_ERR_INVALID_ARG, "n_tensors=%d n_bits=%d n_iters=%d n_restarts=%d", n_tensors, n_bits, n_iters,
+                    n_restarts);
+    if (!mse_table || !n_params || !bits || !t_init || !bits_out || !result)
+        return fail(WQ_ERR_INVALID_ARG, "NULL pointer");
+    for (int j = 0; j < n_bits; ++j)
+        if (bits[j] < 1 || bits[j] > 16 || (j > 0 && bits[j] <= bits[j - 1]))
+            return fail(WQ_ERR_INVALID_ARG, "candidate widths must be strictly increasing in 1..16");
+    for (int i = 0; i < n_tensors; ++i)
+        if (n_params[i] <= 0) return fail(WQ_ERR_INVALID_ARG, "tensor %d: n_params=%lld", i, (long long)n_params[i]);
+    for (int64_t k = 0; k < (int64_t)n_tensors * n_bits; ++k)
+        if (!(mse_table[k] >= 0.0) || std::isinf(mse_table[k]))
+            return fail(WQ_ERR_INVALID_ARG, "mse_table[%lld] is not a finite non-negative number", (long long)k);
+    if (!(target_bpw >= bits[0] && target_bpw <= bits[n_bits - 1]))
+        return fail(WQ_ERR_INVALID_ARG, "target_bpw=%g outside the candidate widths", target_bpw);
+    const wq::PdResult r = wq::pd_search_host(mse_table, n_params, n_tensors, bits, n_bits, target_bpw, n_iters,
+                                              n_restarts, t_init, bits_out);
+    result[0] = r.total_mse;
+    result[1] = r.bpw;
+    result[2] = (double)r.restart;
+    return WQ_OK;
 }
 
 size_t wq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits, int rank) {
@@ -658,6 +745,8 @@ wq_status wq_linear_ex(const void *x, int64_t M, int64_t K, const uint8_t *packe
 
     wq::SmallMArgs a{};
     a.x = static_cast<const uint16_t *>(x);
+    a.packed = packed;
+    a.row_bytes = K * bits / 8;
     a.scales = scales;
     a.bias = static_cast<const uint16_t *>(bias);
     a.L2 = static_cast<const uint16_t *>(L2);
@@ -679,11 +768,11 @@ wq_status wq_linear_ex(const void *x, int64_t M, int64_t K, const uint8_t *packe
         a.t = t;
     }
     switch (bits) {
-        case 3: return launch_smallm<3>(a, packed, dev, info->sm_count, st);
-        case 4: return launch_smallm<4>(a, packed, dev, info->sm_count, st);
-        case 5: return launch_smallm<5>(a, packed, dev, info->sm_count, st);
-        case 6: return launch_smallm<6>(a, packed, dev, info->sm_count, st);
-        default: return launch_smallm<7>(a, packed, dev, info->sm_count, st);
+        case 3: return launch_smallm<3>(a, dev, info->sm_count, st);
+        case 4: return launch_smallm<4>(a, dev, info->sm_count, st);
+        case 5: return launch_smallm<5>(a, dev, info->sm_count, st);
+        case 6: return launch_smallm<6>(a, dev, info->sm_count, st);
+        default: return launch_smallm<7>(a, dev, info->sm_count, st);
     }
 }
 

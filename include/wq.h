@@ -95,6 +95,18 @@ WQ_API int64_t wq_scales_count(int64_t N, int64_t K, int group);
 WQ_API wq_status wq_quantize_pack(const void *W, int64_t N, int64_t K, int bits, int group,
                            uint8_t *packed, float *scales, wq_stream_t stream);
 
+/*
+ * Dequantize a packed weight to bf16 ([PG] sec. 3.4, dequantize_on_gpu: the step before the
+ * page's bf16 matmul):  W_hat[n][k] = bf16(fl32((code - 2^(bits-1)) * step[n][k/128])),
+ * rounded to nearest even.
+ *   packed, scales in : as wq_quantize_pack writes them (N x K*bits/8 bytes, N x K/128 fp32).
+ *   W_hat         out : N x K bf16, row-major.
+ * K must be a multiple of group (128). N == 0 is a no-op. wq_linear does not need this: it
+ * dequantizes in registers; the call is for callers that want the weight itself.
+ */
+WQ_API wq_status wq_dequantize(const uint8_t *packed, const float *scales, int64_t N, int64_t K, int bits,
+                               int group, void *W_hat, wq_stream_t stream);
+
 /* One tensor of a wq_quantize_pack_many call: the arguments of one wq_quantize_pack. */
 typedef struct {
     const void *W;        /* N x K bf16, device */
@@ -119,6 +131,54 @@ typedef struct {
  * launches before it have been queued.
  */
 WQ_API wq_status wq_quantize_pack_many(const wq_pack_job *jobs, int n_jobs, int group, wq_stream_t stream);
+
+/*
+ * Quantization error table of one weight ([PG] sec. 3.2: the per-tensor error at every
+ * candidate width that the PD bit allocation minimizes, its mse_table):
+ *   out[b - 3] = sum over all N*K weights of (w - dequant(quantize_b(w)))^2, for b = 3..7,
+ *   out[5]     = sum of w^2,
+ * where quantize_b / dequant are exactly those of wq_quantize_pack at b bits and wq_linear's
+ * dequant(code) = q * step (fp32). So out[b-3] / (N*K) is the tensor's MSE at b bits and
+ * 10 log10(out[5] / out[b-3]) its SNR in dB.
+ *   W   in : N x K bf16, row-major, finite. K a multiple of group; group must be 128.
+ *   out out: device array of 6 doubles (8-byte aligned), overwritten.
+ * The squared errors are summed in fp64; the order of the final additions varies between
+ * runs, so the last bits of a sum may too. N == 0 writes zeros.
+ */
+WQ_API wq_status wq_quant_error(const void *W, int64_t N, int64_t K, int group, double *out, wq_stream_t stream);
+
+/* One tensor of a wq_quant_error_many call: the arguments of one wq_quant_error. */
+typedef struct {
+    const void *W;        /* N x K bf16, device */
+    int64_t N, K;         /* K a multiple of 128 */
+    double *out;          /* 6 doubles, device */
+} wq_error_job;
+
+/* The error table of many tensors (a whole model) in a few launches (up to 64 tensors each).
+ * Every job is checked before anything is launched; outputs must not overlap. */
+WQ_API wq_status wq_quant_error_many(const wq_error_job *jobs, int n_jobs, int group, wq_stream_t stream);
+
+/*
+ * Per-tensor bit-width search ([PG] sec. 3.2, PD-guided mixed precision), on the host: choose
+ * one width per tensor from `bits` that minimizes the weight-averaged quantization MSE with
+ * a bits-per-weight budget. The relaxation (sigmoid-mapped continuous widths, softmax soft
+ * assignment at a temperature annealed from 2 to 0.05, Lagrange term from 0.5 plus a 1e4
+ * quadratic penalty, n_iters steps from each of n_restarts starts, rounding to the nearest
+ * candidate, best start kept) is described with its readings in the library source.
+ *   mse_table  in : n_tensors x n_bits, row-major, host: per-weight MSE of tensor i at
+ *                   bits[j] (wq_quant_error's sums divided by N*K).
+ *   n_params   in : n_tensors weight counts, host.
+ *   bits       in : n_bits candidate widths, strictly increasing (e.g. 3,4,5,6,7), host.
+ *   t_init     in : n_restarts x n_tensors starting parameters, host (the page draws them
+ *                   as randn * 0.5); the search is deterministic given them.
+ *   bits_out  out : n_tensors chosen widths, host.
+ *   result    out : 3 doubles, host: the choice's total MSE (weight-averaged), its BPW, and
+ *                   the index of the start it came from.
+ * Runs synchronously on the calling thread; touches no GPU.
+ */
+WQ_API wq_status wq_pd_search(const double *mse_table, const int64_t *n_params, int n_tensors, const int *bits,
+                              int n_bits, double target_bpw, int n_iters, int n_restarts, const double *t_init,
+                              int *bits_out, double *result);
 
 /* Workspace bytes wq_linear / wq_linear_ex need for these sizes on any path
  * (0 if none; the caller then may pass NULL). */

@@ -106,6 +106,13 @@ def dequant(codes, scales, bits, group=128):
     return out
 
 
+def dequant_bf16(codes, scales, bits, group=128):
+    """The dequantized weight as the page's bf16 matmul sees it (Per-group(128) article,
+    sec. 3.4 then 5.3): bf16(fl32(q * step)), round to nearest even. Returns uint16 bf16 bits."""
+    d = dequant(codes, scales, bits, group).view(np.uint32).astype(np.uint64)
+    return ((d + 0x7FFF + ((d >> 16) & 1)) >> 16).astype(np.uint16)
+
+
 def linear_rows(x_bits, deq, L1_bits=None, L2_bits=None, bias_bits=None, rows=None):
     """fp64 y = x deq^T + (x L1) L2 + bias for the selected token rows.
 

@@ -24,13 +24,26 @@ def bf16_f64(bits):
     return synth.bf16_bits_to_f32(bits).astype(np.float64)
 
 
+def bf16_half_ulp(v):
+    """Half a unit in the last place of bf16 (8 significant bits) at the magnitude of v: the
+    largest error of a correctly rounded bf16 value there."""
+    a = np.abs(np.asarray(v, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -140)))
+    return 2.0 ** (np.maximum(e, -126.0) - 8.0)
+
+
 def linear_error(y_bits, y_ref):
-    """(relative Frobenius error, max |err| / rms(y_ref)) of a bf16 result vs fp64 reference."""
+    """(relative Frobenius error, max excess error / rms(y_ref)) of a bf16 result vs the fp64
+    reference. The layer's output is bf16 (one rounding of acc + bias), so the max bar
+    measures each element's error beyond its own correct rounding: |y - y_ref| minus half a
+    bf16 ulp at that element. (A correctly rounded output alone reaches 2e-2 rms wherever an
+    element is ~5x the rms or more.) The Frobenius error is the plain one."""
     y = bf16_f64(y_bits)
-    err = y - y_ref
+    err = np.abs(y - y_ref)
     rms = float(np.sqrt(np.mean(y_ref ** 2)))
-    rel = float(np.linalg.norm(err) / max(np.linalg.norm(y_ref), 1e-300))
-    return rel, float(np.abs(err).max() / max(rms, 1e-300))
+    rel = float(np.linalg.norm(y - y_ref) / max(np.linalg.norm(y_ref), 1e-300))
+    excess = np.maximum(err - bf16_half_ulp(np.maximum(np.abs(y), np.abs(y_ref))), 0.0)
+    return rel, float(excess.max() / max(rms, 1e-300))
 
 
 def assert_linear_close(y_bits, y_ref, what=""):

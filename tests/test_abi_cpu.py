@@ -29,7 +29,7 @@ def header_functions():
 
 def test_exports_match_header(L):
     declared = header_functions()
-    assert len(declared) == 14
+    assert len(declared) == 18
     out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
     exported = sorted(line.split()[-1] for line in out.splitlines() if line.split()[-1].startswith("wq_"))
@@ -67,7 +67,7 @@ def test_scope_signatures_match_header(tmp_path):
     assert r.returncode == 0, r.stderr
 
 
-_CTYPES = {"int64_t": ctypes.c_int64, "int": ctypes.c_int, "size_t": ctypes.c_size_t,
+_CTYPES = {"double": ctypes.c_double, "int64_t": ctypes.c_int64, "int": ctypes.c_int, "size_t": ctypes.c_size_t,
            "uint32_t": ctypes.c_uint32, "uint64_t": ctypes.c_uint64, "wq_status": ctypes.c_int,
            "wq_path": ctypes.c_int, "wq_stream_t": ctypes.c_void_p}
 
@@ -80,7 +80,8 @@ def _ctype_of(decl):
         return ctypes.c_char_p
     if "*" in decl:
         base = decl.split("*")[0].strip()
-        return ctypes.POINTER(B.PackJob) if base == "wq_pack_job" else ctypes.c_void_p
+        structs = {"wq_pack_job": B.PackJob, "wq_error_job": B.ErrorJob}
+        return ctypes.POINTER(structs[base]) if base in structs else ctypes.c_void_p
     return _CTYPES[decl.split()[0]]
 
 
@@ -181,6 +182,33 @@ def test_pack_job_struct_matches_header(tmp_path):
     P = B.PackJob
     assert got == [ctypes.sizeof(P), P.W.offset, P.N.offset, P.K.offset, P.bits.offset, P.packed.offset,
                    P.scales.offset]
+
+
+def test_error_job_struct_matches_header(tmp_path):
+    """The binding's ErrorJob has the size and field offsets of the C wq_error_job."""
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "wq.h"\n'
+        'int main(void) { printf("%zu %zu %zu %zu %zu\\n", sizeof(wq_error_job), offsetof(wq_error_job, W),'
+        ' offsetof(wq_error_job, N), offsetof(wq_error_job, K), offsetof(wq_error_job, out)); return 0; }\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    E = B.ErrorJob
+    assert got == [ctypes.sizeof(E), E.W.offset, E.N.offset, E.K.offset, E.out.offset]
+
+
+def test_quant_error_argument_checks(L):
+    A = 0x10000          # aligned fake addresses; none of these calls gets past the checks
+    v = ctypes.c_void_p
+    assert L.wq_quant_error(v(A), 4, 128, 64, v(A), None) == B.WQ_ERR_UNSUPPORTED_GROUP
+    assert L.wq_quant_error(v(A), 4, 130, 128, v(A), None) == B.WQ_ERR_INVALID_ARG
+    assert L.wq_quant_error(v(A), -1, 128, 128, v(A), None) == B.WQ_ERR_INVALID_ARG
+    assert L.wq_quant_error(v(A), 4, 128, 128, None, None) == B.WQ_ERR_INVALID_ARG
+    assert L.wq_quant_error(v(A + 8), 4, 128, 128, v(A), None) == B.WQ_ERR_MISALIGNED
+    assert L.wq_quant_error(v(A), 4, 128, 128, v(A + 4), None) == B.WQ_ERR_MISALIGNED
+    assert L.wq_quant_error_many(None, 3, 128, None) == B.WQ_ERR_INVALID_ARG
+    assert L.wq_quant_error_many(None, 0, 128, None) == B.WQ_OK
 
 
 def test_quantize_pack_many_argument_checks(L):
