@@ -14,13 +14,13 @@
 //
 // Orientation: D = W_q x^T, so TMEM lanes are weight rows and columns are tokens; the
 // per-group step is then one scalar per lane.
-// One persistent CTA per SM walks tiles of 128 weight rows x TT tokens (TT = 256, or 128 for
-// few tokens), weight tiles fastest, so a wave of CTAs shares one token tile of x in L2 and
+// One persistent CTA per SM walks tiles of 128 weight rows x TT tokens (TT = 256 or 240,
+// whichever leaves the last wave of tiles fuller, or 128 for few tokens), weight tiles fastest, so a wave of CTAs shares one token tile of x in L2 and
 // the (4-8x smaller) packed weight stays L2-resident across token tiles.
 // Shared memory: a ring of kStages 64-k stages, each holding the x tile (TT tokens x 64 k,
 // bf16, 128-byte swizzle, by TMA) and the code tile (128 rows x 64 k exact bf16 q, the same
-// swizzled layout, written by the unpack warps). TMEM (512 columns): T0, T1 = the per-group
-// partial products (double-buffered, TT columns each).
+// swizzled layout, written by the unpack warps). TMEM (512 columns): T0 at column 0 and T1 at
+// column 256 = the per-group partial products (double-buffered, TT columns each).
 // One unit = one 128-k group (two stages) or the low-rank unit. Per unit, one MMA-issuing
 // thread waits for T to be free and for each stage to be full, issues M=128 N=TT K=16 MMAs
 // (A = codes, B = x, both from shared memory), releases each stage with a commit and hands T
@@ -63,7 +63,7 @@ static_assert(kTcRegsWg0 + kTcRegsWg1 + 2 * kTcRegsPromote == 4 * kTcRegsLaunch,
 
 template <int TT>
 struct TcLayout {
-    static constexpr int kStages = TT == 256 ? 4 : 6;
+    static constexpr int kStages = TT > 128 ? 4 : 6;
     static constexpr uint32_t kXBytes = TT * kTcBK * 2;             // 32 KB (TT = 256)
     static constexpr uint32_t kABytes = kTcBW * kTcBK * 2;          // 16 KB
     static constexpr uint32_t kOffX = 0;
@@ -216,14 +216,18 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
             int armed[S];
             for (int i = 0; i < S; ++i) armed[i] = -1;
             int l_armed = -1;
-            uint32_t q = 0, lph = 0;
+            // p_full[s] is armed only when stage s is a group's second stage, which is not every
+            // use of s (a one-stage low-rank unit shifts the pairing), so its phase is counted
+            // per stage: bit s of pph
+            uint32_t q = 0, lph = 0, pph = 0;
             for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
                 const int nt = tile % p.tiles_n;
                 for (int u = 0; u < G; ++u, q += 2) {
                     const uint32_t s1 = (q + 1) % S, ph1 = ((q + 1) / S) & 1;
                     if (!mbar_wait(&empty[s1], ph1 ^ 1, abort)) goto p_done;
                     mbar_arrive_expect_tx(&p_full[s1], (uint32_t)kTcBW * 16u * BITS);
-                    armed[s1] = (int)ph1;
+                    armed[s1] = (int)((pph >> s1) & 1u);
+                    pph ^= 1u << s1;
                     tma_load_2d(smem + L::kOffA + s1 * L::kABytes, &p_map, &p_full[s1], u * 16 * BITS, nt * kTcBW);
                 }
                 if (p.rank > 0) {
@@ -260,7 +264,7 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                     const uint32_t tb = unit & 1;
                     if (!mbar_wait(&t_empty[tb], ((unit >> 1) & 1) ^ 1, abort)) goto m_done;
                     tc_fence_after();
-                    const uint32_t d = tmem + tb * TT;
+                    const uint32_t d = tmem + tb * 256u;
                     for (int st = 0; st < nst; ++st, ++q) {
                         const uint32_t s = q % S, ph = (q / S) & 1;
                         if (!mbar_wait(&full[s], ph, abort)) goto m_done;
@@ -288,17 +292,18 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         // ---------------------------------------------------------- unpack codes into shared memory
         const int row_local = threadIdx.x - 128;
         const uint32_t a_base = smem_u32(smem + L::kOffA);
-        uint32_t q = 0, lph = 0;
+        uint32_t q = 0, lph = 0, pph = 0;     // pph: per-stage phase bits of p_full (see the producer)
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int nt = tile % p.tiles_n;
             const int64_t n = (int64_t)nt * kTcBW + row_local;
             const bool row_ok = n < p.N;        // (rows past N arrive as zeros and are never stored)
             for (int g = 0; g < G; ++g) {
                 const uint32_t s0 = q % S, ph0 = (q / S) & 1;
-                const uint32_t s1 = (q + 1) % S, ph1 = ((q + 1) / S) & 1;
+                const uint32_t s1 = (q + 1) % S;
                 q += 2;
                 // this row's packed group, from the tile the producer put in stage s1's code buffer
-                const bool got = warp_wait(&p_full[s1], ph1, abort);
+                const bool got = warp_wait(&p_full[s1], (pph >> s1) & 1u, abort);
+                pph ^= 1u << s1;
                 uint32_t w[NWG];
                 w[4 * BITS] = 0;
                 if (got) {
@@ -403,13 +408,22 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                 const uint32_t tb = unit & 1, tph = (unit >> 1) & 1;
                 if (!warp_wait(&t_full[tb], tph, abort)) goto pr_done;
                 tc_fence_after();
-                const uint32_t t_addr = tmem + lane_addr + tb * TT + colh * kHalf;
-#pragma unroll
-                for (int hf = 0; hf < kHalf / 32; ++hf) {
+                const uint32_t t_addr = tmem + lane_addr + tb * 256u + colh * kHalf;
+                // this warp's kHalf columns in chunks of 32 (then one chunk of the remaining
+                // multiple of 8); T is handed back once the last chunk is in registers
+                constexpr int kFull = kHalf / 32, kRest = kHalf % 32, kChunks = kFull + (kRest ? 1 : 0);
+                static_for<kChunks>([&](auto hc) {
+                    constexpr int hf = decltype(hc)::value;
+                    constexpr int width = hf < kFull ? 32 : kRest;
                     uint32_t tv[32];
-                    tmem_ld_32x32b_x32(t_addr + 32 * hf, tv);
+                    if constexpr (width == 32) {
+                        tmem_ld_32x32b_x32(t_addr + 32 * hf, tv);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < width / 8; ++e) tmem_ld_32x32b_x8(t_addr + 32 * hf + 8 * e, tv + 8 * e);
+                    }
                     tmem_wait_ld();
-                    if (hf == kHalf / 32 - 1) {
+                    if (hf == kChunks - 1) {
                         // all of this warp's T columns are in registers: hand the buffer back
                         tc_fence_before();
                         __syncwarp();
@@ -417,14 +431,14 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
                     }
                     if (u == 0) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) R[32 * hf + i] = __uint_as_float(tv[i]) * s;
+                        for (int i = 0; i < width; ++i) R[32 * hf + i] = __uint_as_float(tv[i]) * s;
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2)
+                        for (int i = 0; i < width; i += 2)
                             ffma2(R[32 * hf + i], R[32 * hf + i + 1], __uint_as_float(tv[i]), __uint_as_float(tv[i + 1]),
                                   s, s, R[32 * hf + i], R[32 * hf + i + 1]);
                     }
-                }
+                });
             }
             // ------------------------------------------------------ epilogue
             if (row_ok) {

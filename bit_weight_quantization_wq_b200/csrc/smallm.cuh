@@ -160,20 +160,35 @@ smallm_kernel(const SmallMArgs a) {
     const int gs0 = shared_blocks ? Gc * split / a.GW : 0, gs1 = shared_blocks ? Gc * (split + 1) / a.GW : Gc;
 
     // The copies of one item: 16 rows x 16*b bytes of codes (16-byte copies, rows past N
-    // zero-filled) and the 16 rows' steps (4-byte copies) into ring slot `slot`.
+    // zero-filled) and the 16 rows' steps (4-byte copies) into ring slot `slot`. Which chunks
+    // a lane copies does not change between items, so their row and offsets are computed
+    // once; an item only moves the base address.
+    constexpr int kChunkIters = (16 * BITS + 31) / 32;
+    int c_row[kChunkIters];
+    int64_t c_src[kChunkIters];
+    uint32_t c_dst[kChunkIters];
+#pragma unroll
+    for (int i = 0; i < kChunkIters; ++i) {
+        const int j = lane + 32 * i;
+        const int row = j / BITS, ch = j - row * BITS;
+        c_row[i] = j < 16 * BITS ? row : 1 << 30;             // lanes without an i-th chunk
+        c_src[i] = (int64_t)row * a.row_bytes + 16 * ch;
+        c_dst[i] = (uint32_t)row * kGB + 16u * ch;
+    }
+    const int64_t step_src = (int64_t)lane * G;
     auto issue = [&](int64_t n0, int g, uint32_t slot) {
-        const uint8_t *base = a.packed + (int64_t)g * kGB;
-        for (int j = lane; j < 16 * BITS; j += 32) {
-            const int row = j / BITS, ch = j - row * BITS;
-            const int64_t n = n0 + row;
-            const bool ok = n < a.N;
-            cp_async_16(slot + (uint32_t)row * kGB + 16u * ch, ok ? base + n * a.row_bytes + 16 * ch : a.packed,
-                        ok ? 16u : 0u);
+        const uint8_t *base = a.packed + n0 * a.row_bytes + (int64_t)g * kGB;
+        const int64_t rows_left = a.N - n0;
+#pragma unroll
+        for (int i = 0; i < kChunkIters; ++i) {
+            if (c_row[i] < 16) {
+                const bool ok = c_row[i] < rows_left;
+                cp_async_16(slot + c_dst[i], ok ? base + c_src[i] : a.packed, ok ? 16u : 0u);
+            }
         }
         if (lane < 16) {
-            const int64_t n = n0 + lane;
-            const bool ok = n < a.N;
-            cp_async_4(slot + 16u * kGB + 4u * lane, ok ? a.scales + n * G + g : a.scales, ok ? 4u : 0u);
+            const bool ok = lane < rows_left;
+            cp_async_4(slot + 16u * kGB + 4u * lane, ok ? a.scales + n0 * G + step_src + g : a.scales, ok ? 4u : 0u);
         }
     };
     // A segment walks its items group-major: (group gs0, unit 0..nr-1), (gs0 + 1, ...), ...

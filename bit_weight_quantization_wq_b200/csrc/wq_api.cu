@@ -410,8 +410,9 @@ wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &t
 template <int BITS>
 wq_status launch_tc_tt(const TcArgs &a, int tt, const CUtensorMap &xm, const CUtensorMap &tm, const CUtensorMap &lm,
                        const CUtensorMap &pm, int l_tma, int sm_count, cudaStream_t st) {
-    return tt == 256 ? launch_tc<BITS, 256>(a, xm, tm, lm, pm, l_tma, sm_count, st)
-                     : launch_tc<BITS, 128>(a, xm, tm, lm, pm, l_tma, sm_count, st);
+    if (tt == 256) return launch_tc<BITS, 256>(a, xm, tm, lm, pm, l_tma, sm_count, st);
+    if (tt == 240) return launch_tc<BITS, 240>(a, xm, tm, lm, pm, l_tma, sm_count, st);
+    return launch_tc<BITS, 128>(a, xm, tm, lm, pm, l_tma, sm_count, st);
 }
 
 template <int R>
@@ -449,16 +450,30 @@ wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_
     return check_launch("lowrank_prepass_kernel");
 }
 
-// Tokens per tensor-core tile: 256 (one MMA covers 128 weight rows x 256 tokens, which hides
-// the per-group hand-off of the partial products), 128 when there are few tokens.
-int tc_tile_tokens(int64_t M) { return M > 128 ? 256 : 128; }
+// Tokens per tensor-core tile: 256 or 240 (one MMA covers 128 weight rows x that many tokens,
+// long enough to hide the per-group hand-off of the partial products), whichever needs fewer
+// tile-waves x tokens on this many SMs (a last wave left mostly empty costs a whole wave); 128
+// when there are few tokens.
+int tc_tile_tokens(int64_t M, int64_t N, int sm_count) {
+    if (M <= 128) return 128;
+    const int64_t tiles_n = (N + wq::kTcBW - 1) / wq::kTcBW;
+    int best = 256;
+    int64_t best_cost = -1;
+    for (int tt : {256, 240}) {
+        const int64_t tiles = (M + tt - 1) / tt * tiles_n;
+        const int64_t waves = (tiles + sm_count - 1) / sm_count;
+        const int64_t cost = waves * tt;
+        if (best_cost < 0 || cost < best_cost) { best = tt; best_cost = cost; }
+    }
+    return best;
+}
 
 wq_status tc_linear(const TcArgs &a, int sm_count, cudaStream_t st) {
     wq_status s = get_encoder();
     if (s != WQ_OK) return s;
     if (a.M > (int64_t)INT32_MAX || a.N > (int64_t)INT32_MAX || a.K > (int64_t)INT32_MAX)
         return fail(WQ_ERR_INVALID_ARG, "dimension above 2^31 on the tensor-core path");
-    const int tt = tc_tile_tokens(a.M);
+    const int tt = tc_tile_tokens(a.M, a.N, sm_count);
     CUtensorMap xm, tm, lm;
     int l_tma = 0;
     if ((s = make_map_2d(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)a.K, (uint64_t)a.M,
