@@ -467,80 +467,104 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
 // t = x L1 (M x R, R = rank 16..64) as two bf16 terms, t_hi = bf16(t) in columns [0, R) and
 // t_lo = bf16(t - t_hi) in [R, 2R), row stride kTStride = 128 (the rest zero), so that
 // 64-wide TMA boxes cover a row exactly.
-// x is read once; tensor cores via mma.m16n8k16.
-// grid (ceil(M/64), KS) with clusters of KS CTAs along K; a CTA owns 64 tokens (4 warps x
-// 16) and 1/KS of K; partial sums are added through distributed shared memory.
+// x is read once, at close to HBM rate; tensor cores via mma.m16n8k16.
+// grid (ceil(M/64), KS) with clusters of KS (<= 16) CTAs along K; a CTA owns 64 tokens (4
+// warps x 16) and 1/KS of K. Its share of L1 (K/KS x R bf16) is copied into shared memory in
+// passes of up to `sb` 64-k blocks (all of it at once when it fits), x is streamed from global
+// memory kPrePf blocks ahead in registers, and the KS partial sums are added through
+// distributed shared memory.
 // Inside a thread, k is taken in the order that makes its x loads contiguous (16
-// consecutive k per row per 64-k stage); the L1 fragments are fetched with
-// ldmatrix.trans from row addresses in the same order.
+// consecutive k per row per 64-k block); the L1 fragments are fetched with ldmatrix.trans
+// from row addresses in the same order.
+constexpr int kPreMaxKS = 16;
+constexpr int kPrePf = 3;                               // x blocks in flight per thread
+
+// shared memory of a prepass CTA staging `sb` 64-k blocks of L1 at a time
+template <int R>
+__host__ __device__ constexpr uint32_t prepass_smem_bytes(int sb) {
+    return (uint32_t)sb * 64u * (R + 8) * 2u + 64u * R * 4u;
+}
+
 template <int R>
 __global__ void __launch_bounds__(128)
 lowrank_prepass_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ L1,
-                       uint16_t *__restrict__ t, int64_t M, int64_t K) {
+                       uint16_t *__restrict__ t, int64_t M, int64_t K, int sb) {
     constexpr int kLd = R + 8;                          // padded smem row (elements)
-    __shared__ __align__(16) uint16_t l1s[2][64 * kLd];
-    __shared__ __align__(16) float part[64 * R];
+    extern __shared__ __align__(16) uint8_t pre_smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
     const uint32_t KS = gridDim.y, split = cluster_ctarank();
     const int64_t m0 = (int64_t)blockIdx.x * 64;
     const int64_t nkb = K / 64;
     const int64_t kb0 = nkb * split / KS, kb1 = nkb * (split + 1) / KS;
+    const int nb = (int)(kb1 - kb0);
+    uint16_t *l1s = reinterpret_cast<uint16_t *>(pre_smem);                   // [sb*64][kLd]
+    float *part = reinterpret_cast<float *>(pre_smem + (size_t)sb * 64 * kLd * 2); // [64][R]
     const int64_t ra = m0 + warp * 16 + g, rb = ra + 8;
+
+    // blocks [b0, b1) of this CTA's share of L1 -> shared memory (asynchronous 16-byte copies)
+    auto stage_l1 = [&](int b0, int b1) {
+        constexpr int per_row = R / 8;                  // 16-byte chunks per L1 row
+        const int chunks = (b1 - b0) * 64 * per_row;
+        for (int i = tid; i < chunks; i += 128) {
+            const int kr = i / per_row, cj = i - kr * per_row;
+            const uint32_t dst = smem_u32(l1s + kr * kLd + cj * 8);
+            const uint16_t *src = L1 + ((kb0 + b0) * 64 + kr) * R + cj * 8;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    auto load_x = [&](int64_t kb, uint4 (&xa)[2], uint4 (&xb)[2]) {
+        const int64_t k = kb * 64 + 16 * c;
+        if (ra < M) { xa[0] = ldg_stream_v4(x + ra * K + k); xa[1] = ldg_stream_v4(x + ra * K + k + 8); }
+        else xa[0] = xa[1] = make_uint4(0, 0, 0, 0);
+        if (rb < M) { xb[0] = ldg_stream_v4(x + rb * K + k); xb[1] = ldg_stream_v4(x + rb * K + k + 8); }
+        else xb[0] = xb[1] = make_uint4(0, 0, 0, 0);
+    };
+    uint4 xa[kPrePf][2], xb[kPrePf][2];
+#pragma unroll
+    for (int p = 0; p < kPrePf; ++p)
+        if (p < nb) load_x(kb0 + p, xa[p], xb[p]);
     float acc[R / 8][4];
 #pragma unroll
     for (int j = 0; j < R / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
 
-    auto load_l1 = [&](int buf, int64_t kb) {
-        constexpr int chunks = 64 * R / 8;              // 16-byte chunks of the 64 x R slab
-        for (int i = tid; i < chunks; i += 128) {
-            const int kr = i / (R / 8), cj = i % (R / 8);
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(L1 + (kb * 64 + kr) * R) + cj);
-            *reinterpret_cast<uint4 *>(&l1s[buf][kr * kLd + cj * 8]) = v;
+    int staged0 = 0, staged1 = 0;                       // L1 blocks [staged0, staged1) are in l1s
+    for (int i0 = 0; i0 < nb; i0 += kPrePf) {
+        if (i0 >= staged1) {
+            // next pass of L1 (sb is a multiple of kPrePf, so a pass starts at an i0)
+            __syncthreads();
+            staged0 = i0;
+            staged1 = min(i0 + sb, nb);
+            stage_l1(staged0, staged1);
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            __syncthreads();
         }
-    };
-    auto load_x = [&](int64_t kb, uint4 (&xa)[2], uint4 (&xb)[2]) {
-        const int64_t k = kb * 64 + 16 * c;
-        if (ra < M) { xa[0] = __ldg(reinterpret_cast<const uint4 *>(x + ra * K + k)); xa[1] = __ldg(reinterpret_cast<const uint4 *>(x + ra * K + k + 8)); }
-        else xa[0] = xa[1] = make_uint4(0, 0, 0, 0);
-        if (rb < M) { xb[0] = __ldg(reinterpret_cast<const uint4 *>(x + rb * K + k)); xb[1] = __ldg(reinterpret_cast<const uint4 *>(x + rb * K + k + 8)); }
-        else xb[0] = xb[1] = make_uint4(0, 0, 0, 0);
-    };
-
-    uint4 xa[2], xb[2], na[2], nb[2];
-    if (kb0 < kb1) {
-        load_l1(0, kb0);
-        load_x(kb0, xa, xb);
-    }
-    __syncthreads();
-    for (int64_t kb = kb0; kb < kb1; ++kb) {
-        const int buf = (int)((kb - kb0) & 1);
-        if (kb + 1 < kb1) {
-            load_l1(buf ^ 1, kb + 1);
-            load_x(kb + 1, na, nb);
-        }
-        const uint32_t aw[8] = {xa[0].x, xa[0].y, xa[0].z, xa[0].w, xa[1].x, xa[1].y, xa[1].z, xa[1].w};
-        const uint32_t bw[8] = {xb[0].x, xb[0].y, xb[0].z, xb[0].w, xb[1].x, xb[1].y, xb[1].z, xb[1].w};
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            // k-slot q of this step <-> actual k = 16 (q%8 / 2) + 4 s + 2 (q / 8) + (q % 2)
-            const int q = lane & 15;
-            const int kr = 16 * ((q & 7) >> 1) + 4 * s + 2 * (q >> 3) + (q & 1);
+        for (int p = 0; p < kPrePf; ++p) {
+            const int i = i0 + p;
+            if (i >= nb) break;
+            const uint32_t aw[8] = {xa[p][0].x, xa[p][0].y, xa[p][0].z, xa[p][0].w, xa[p][1].x, xa[p][1].y, xa[p][1].z, xa[p][1].w};
+            const uint32_t bw[8] = {xb[p][0].x, xb[p][0].y, xb[p][0].z, xb[p][0].w, xb[p][1].x, xb[p][1].y, xb[p][1].z, xb[p][1].w};
+            if (i + kPrePf < nb) load_x(kb0 + i + kPrePf, xa[p], xb[p]);
+            const uint16_t *l1b = l1s + (size_t)(i - staged0) * 64 * kLd;
 #pragma unroll
-            for (int jt = 0; jt < R / 8; jt += 2) {
-                uint32_t b0, b1, b2, b3;
-                const int col = jt * 8 + (lane >> 4) * 8;
-                const uint32_t addr = smem_u32(&l1s[buf][kr * kLd + (col < R ? col : jt * 8)]);
-                asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                             : "=r"(b0), "=r"(b1), "=r"(b2), "=r"(b3) : "r"(addr));
-                mma_16816_bf16(acc[jt], aw[2 * s], bw[2 * s], aw[2 * s + 1], bw[2 * s + 1], b0, b1);
-                if (jt + 1 < R / 8)
-                    mma_16816_bf16(acc[jt + 1], aw[2 * s], bw[2 * s], aw[2 * s + 1], bw[2 * s + 1], b2, b3);
+            for (int s = 0; s < 4; ++s) {
+                // k-slot q of this step <-> actual k = 16 (q%8 / 2) + 4 s + 2 (q / 8) + (q % 2)
+                const int q = lane & 15;
+                const int kr = 16 * ((q & 7) >> 1) + 4 * s + 2 * (q >> 3) + (q & 1);
+#pragma unroll
+                for (int jt = 0; jt < R / 8; jt += 2) {
+                    uint32_t b0, b1, b2, b3;
+                    const int col = jt * 8 + (lane >> 4) * 8;
+                    const uint32_t addr = smem_u32(l1b + kr * kLd + (col < R ? col : jt * 8));
+                    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                                 : "=r"(b0), "=r"(b1), "=r"(b2), "=r"(b3) : "r"(addr));
+                    mma_16816_bf16(acc[jt], aw[2 * s], bw[2 * s], aw[2 * s + 1], bw[2 * s + 1], b0, b1);
+                    if (jt + 1 < R / 8)
+                        mma_16816_bf16(acc[jt + 1], aw[2 * s], bw[2 * s], aw[2 * s + 1], bw[2 * s + 1], b2, b3);
+                }
             }
-        }
-        __syncthreads();
-        if (kb + 1 < kb1) {
-            xa[0] = na[0]; xa[1] = na[1]; xb[0] = nb[0]; xb[1] = nb[1];
         }
     }
     // partial sums -> shared memory [token][j]
@@ -558,8 +582,16 @@ lowrank_prepass_kernel(const uint16_t *__restrict__ x, const uint16_t *__restric
     const int e0 = (int)((int64_t)E * split / KS), e1 = (int)((int64_t)E * (split + 1) / KS);
     const uint32_t base = smem_u32(part);
     for (int e = e0 + tid; e < e1; e += 128) {
+        // the KS partials in rank order, loaded four at a time
         float v = 0.0f;
-        for (uint32_t r = 0; r < KS; ++r) v += ld_cluster_f32(map_cluster_smem(base + 4u * e, r));
+        for (int r0 = 0; r0 < (int)KS; r0 += 4) {
+            float pv[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                pv[r] = r0 + r < (int)KS ? ld_cluster_f32(map_cluster_smem(base + 4u * e, (uint32_t)(r0 + r))) : 0.0f;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) v += pv[r];
+        }
         const int64_t m = m0 + e / R;
         if (m < M) {
             // two bf16 terms: t_hi = bf16(t) in column j, t_lo = bf16(t - t_hi) in column R + j

@@ -11,24 +11,24 @@
 // contiguous range of units, balanced to +-1 unit over the clusters; its CTAs split the K
 // groups. Inside a CTA each warp owns a block of up to four units and a range of the CTA's
 // groups (when there are fewer blocks than warps, several warps share a block, each with its
-// own groups), and walks its (group, unit) items group-major, so the x fragment of a group is
-// loaded once for all units of the block.
+// own groups), and walks it one group at a time: the x fragment of a group is loaded once
+// for all units of the block, and the units' MMA chains are independent, so they interleave.
 //
-// Data movement: every warp streams its own items. Each item (16 rows x one group of codes,
-// 16*b bytes a row, plus the 16 rows' steps) is copied with 16-byte (and 4-byte)
-// asynchronous copies into a private ring of D slots in shared memory, D - 1 items ahead of
-// the one being computed; the warp waits on its own copy groups only. There is no producer
-// warp and no barrier between warps until the final reduction, so each warp's loads and
-// arithmetic overlap independently. x for the CTA's groups is copied into shared memory once,
-// at the start, with a padded token stride.
+// Data movement: every warp streams its own groups. One ring slot holds one group of the
+// block (16 rows x 16*b bytes per unit), copied with 16-byte asynchronous copies into a
+// private ring of D slots in shared memory, D - 1 groups ahead of the one being computed;
+// the warp waits on its own copy groups only. There is no producer warp and no barrier
+// between warps until the final reduction. At the start the CTA copies into shared memory,
+// once: the token rows of x for its groups (padded stride), every group's sum of x per
+// token, and the steps of all its rows and groups.
 //
 // Arithmetic: thread (g, c) of a warp holds rows g and g+8 of the unit and the 32
 // consecutive codes [32c, 32c+32) of the group, 4*b contiguous bytes per row. Inside one
 // MMA step s the k slots it feeds are mapped to k = 32c + 4s + {0,1} and 32c + 4s + {2,3}
 // (the same map on the x side), so both operands are read in natural order. Codes enter
 // the MMAs as the exact bf16 values 128 + code (bit pattern 0x4300 | code); the group's
-// (128 + 2^(b-1)) * sum(x) is formed by eight more MMAs with a constant A operand and
-// subtracted once per item, which leaves sum_k q x exactly as before rounding. Each
+// (128 + 2^(b-1)) * sum(x), from the per-token group sums computed at the start, is
+// subtracted once per item. Each
 // group's fp32 product is scaled by the group's fp32 step and accumulated in fp32: the
 // weight is never rounded.
 //
@@ -52,7 +52,7 @@ constexpr int kSmMaxRB = 4;                                  // units per warp b
 constexpr int kSmMaxD = 6;                                   // ring slots per warp
 
 template <int TOK> struct SmCfg {
-    static constexpr int kWarps = TOK <= 8 ? 16 : 12;
+    static constexpr int kWarps = 12;
     static constexpr int kThreads = kWarps * 32;
     static constexpr int kNT = TOK / 8;                      // n8 token tiles per MMA step
     static constexpr int kCH = 2;                            // independent MMA accumulators per item
@@ -74,9 +74,10 @@ struct SmallMArgs {
     int RB, GW;               // units per warp block; warps per block (group splits) when blocks < warps
     int D;                    // ring slots per warp (2..kSmMaxD)
     int rows_max;             // rows of the largest cluster range (units * 16)
-    uint32_t x_stride;        // bytes per token row of the staged x (groups * 256 + 64)
-    uint32_t slot_bytes;      // one ring slot: 16 rows x 16b bytes of codes, then 16 fp32 steps
-    uint32_t off_ring, off_part;
+    int gmax;                 // groups of the largest CTA share (row stride of the staged sums and steps)
+    uint32_t x_stride;        // bytes per token row of the staged x (gmax * 256 + 64)
+    uint32_t slot_bytes;      // one ring slot: RB units x 16 rows x 16b bytes of codes
+    uint32_t off_sx, off_st, off_ring, off_part;
 };
 
 // ---------------------------------------------------------------- asynchronous copies
@@ -128,8 +129,7 @@ smallm_kernel(const SmallMArgs a) {
     constexpr int NT = SmCfg<TOK>::kNT;
     constexpr int CH = SmCfg<TOK>::kCH;
     constexpr uint32_t kGB = 16 * BITS;                        // bytes of one group of one row
-    // bf16x2 (128 + 2^(b-1)) in both halves: the bias the unpacked codes carry
-    constexpr uint32_t kBias2 = (uint32_t)(0x4300 + (1 << (BITS - 1))) * 0x10001u;
+    constexpr float kBiasF = 128.0f + (float)(1 << (BITS - 1)); // the bias the unpacked codes carry
     extern __shared__ __align__(128) uint8_t smem[];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -144,10 +144,13 @@ smallm_kernel(const SmallMArgs a) {
     const int g0 = (int)((int64_t)G * srank / S), g1 = (int)((int64_t)G * (srank + 1) / S);
     const int Gc = g1 - g0;
     const int rows_c = Uc * 16;
-    const uint32_t x_base = smem_u32(smem);
-    const uint32_t ring = smem_u32(smem + a.off_ring) + (uint32_t)warp * (uint32_t)a.D * a.slot_bytes;
+    const int64_t n_base = u0 * 16;
+    const int M = (int)a.M;                                     // 1..TOK
+    float *sx = reinterpret_cast<float *>(smem + a.off_sx);     // [TOK][gmax] group sums of x
+    float *st = reinterpret_cast<float *>(smem + a.off_st);     // [rows_max][gmax] steps
     float *part = reinterpret_cast<float *>(smem + a.off_part);
-    const int part_stride = TOK * a.rows_max;                 // floats per group split
+    const int part_stride = TOK * a.rows_max;                   // floats per group split
+    const uint32_t ring = smem_u32(smem + a.off_ring) + (uint32_t)warp * (uint32_t)a.D * a.slot_bytes;
 
     // ---------------------------------------------------------------- this warp's blocks
     const int RB = a.RB;
@@ -159,79 +162,90 @@ smallm_kernel(const SmallMArgs a) {
     const bool active = shared_blocks ? (warp < NB * a.GW) : true;
     const int gs0 = shared_blocks ? Gc * split / a.GW : 0, gs1 = shared_blocks ? Gc * (split + 1) / a.GW : Gc;
 
-    // The copies of one item: 16 rows x 16*b bytes of codes (16-byte copies, rows past N
-    // zero-filled) and the 16 rows' steps (4-byte copies) into ring slot `slot`. Which chunks
-    // a lane copies does not change between items, so their row and offsets are computed
-    // once; an item only moves the base address.
-    constexpr int kChunkIters = (16 * BITS + 31) / 32;
+    // The copies of one slot: group g of the nr units from row n0, 16 rows x 16*b bytes each
+    // (16-byte copies, rows past N zero-filled). Which chunks a lane copies does not change
+    // between slots, so their row and offsets are computed once.
+    constexpr int kChunks = kSmMaxRB * 16 * BITS;              // 16-byte chunks of a full slot
+    constexpr int kChunkIters = (kChunks + 31) / 32;
     int c_row[kChunkIters];
     int64_t c_src[kChunkIters];
     uint32_t c_dst[kChunkIters];
 #pragma unroll
     for (int i = 0; i < kChunkIters; ++i) {
         const int j = lane + 32 * i;
-        const int row = j / BITS, ch = j - row * BITS;
-        c_row[i] = j < 16 * BITS ? row : 1 << 30;             // lanes without an i-th chunk
+        const int row = j / BITS, ch = j - row * BITS;        // row of the slot: unit row / 16
+        c_row[i] = j < kChunks ? row : 1 << 30;
         c_src[i] = (int64_t)row * a.row_bytes + 16 * ch;
         c_dst[i] = (uint32_t)row * kGB + 16u * ch;
     }
-    const int64_t step_src = (int64_t)lane * G;
-    auto issue = [&](int64_t n0, int g, uint32_t slot) {
+    auto issue = [&](int64_t n0, int nr, int g, uint32_t slot) {
         const uint8_t *base = a.packed + n0 * a.row_bytes + (int64_t)g * kGB;
         const int64_t rows_left = a.N - n0;
 #pragma unroll
         for (int i = 0; i < kChunkIters; ++i) {
-            if (c_row[i] < 16) {
+            if (c_row[i] < 16 * nr) {
                 const bool ok = c_row[i] < rows_left;
                 cp_async_16(slot + c_dst[i], ok ? base + c_src[i] : a.packed, ok ? 16u : 0u);
             }
         }
-        if (lane < 16) {
-            const bool ok = lane < rows_left;
-            cp_async_4(slot + 16u * kGB + 4u * lane, ok ? a.scales + n0 * G + step_src + g : a.scales, ok ? 4u : 0u);
-        }
+        cp_async_commit();
     };
-    // A segment walks its items group-major: (group gs0, unit 0..nr-1), (gs0 + 1, ...), ...
-    // The prefetch cursor runs D - 1 items ahead of the item being computed; both move one item
-    // (and one ring slot) at a time, so no index is divided.
-    struct Cursor { int gl, r; uint32_t slot; };
-    auto advance = [&](Cursor &c, int nr) {
-        if (++c.r == nr) { c.r = 0; ++c.gl; }
-        c.slot += a.slot_bytes;
-        if (c.slot == ring + (uint32_t)a.D * a.slot_bytes) c.slot = ring;
-    };
-    auto prologue = [&](int ub, int nr, Cursor &pf) {
-        pf = Cursor{gs0, 0, ring};
-        for (int i = 0; i < a.D - 1; ++i) {
-            if (pf.gl < gs1) {
-                issue((u0 + ub + pf.r) * 16, g0 + pf.gl, pf.slot);
-                advance(pf, nr);
-            }
-            cp_async_commit();
-        }
-    };
+    auto slot_next = [&](uint32_t s) { s += a.slot_bytes; return s == ring + (uint32_t)a.D * a.slot_bytes ? ring : s; };
 
-    // first copies go out before x is staged, so the ring fills while x arrives
+    // first copies go out before the staging, so the ring fills while x arrives
     const int first_ub = shared_blocks ? (warp % NB) * RB : warp * RB;
-    Cursor pf;
-    if (active && first_ub < Uc) prologue(first_ub, min(RB, Uc - first_ub), pf);
+    uint32_t pf_slot = ring;
+    int pf_gl = gs0;
+    auto prologue = [&](int ub, int nr) {
+        pf_slot = ring;
+        pf_gl = gs0;
+        for (int i = 0; i < a.D - 1; ++i) {
+            if (pf_gl < gs1) {
+                issue(n_base + ub * 16, nr, g0 + pf_gl, pf_slot);
+                pf_slot = slot_next(pf_slot);
+                ++pf_gl;
+            } else {
+                cp_async_commit();
+            }
+        }
+    };
+    if (active && first_ub < Uc) prologue(first_ub, min(RB, Uc - first_ub));
 
-    // ---------------------------------------------------------------- stage x (padded rows)
+    // ---------------------------------------------------------------- stage x, steps
     {
         const int chunks = Gc * 16;                            // 16-byte chunks per token row
-        for (int e = threadIdx.x; e < TOK * chunks; e += W * 32) {
+        for (int e = threadIdx.x; e < M * chunks; e += W * 32) {
             const int tok = e / chunks, j = e - tok * chunks;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (tok < a.M) v = ldg_stream_v4(a.x + (int64_t)tok * a.K + (int64_t)g0 * 128 + 8 * j);
+            const uint4 v = ldg_stream_v4(a.x + (int64_t)tok * a.K + (int64_t)g0 * 128 + 8 * j);
             *reinterpret_cast<uint4 *>(smem + (uint32_t)tok * a.x_stride + 16u * j) = v;
         }
+        const int rows_v = (int)min((int64_t)rows_c, a.N - n_base);
+        for (int e = threadIdx.x; e < rows_v * Gc; e += W * 32) {
+            const int i = e / Gc, gl = e - i * Gc;
+            st[i * a.gmax + gl] = __ldg(a.scales + (n_base + i) * G + g0 + gl);
+        }
+    }
+    __syncthreads();
+    // sum of each staged token row over each group (fixed order)
+    for (int e = threadIdx.x; e < M * Gc; e += W * 32) {
+        const int tok = e / Gc, gl = e - tok * Gc;
+        const uint4 *xp = reinterpret_cast<const uint4 *>(smem + (uint32_t)tok * a.x_stride + (uint32_t)gl * 256u);
+        float sum = 0.0f;
+#pragma unroll 4
+        for (int q = 0; q < 16; ++q) {
+            const uint4 v = xp[q];
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) sum += bf16_bits_to_f32(wv[h] & 0xFFFFu) + bf16_bits_to_f32(wv[h] >> 16);
+        }
+        sx[tok * a.gmax + gl] = sum;
     }
     __syncthreads();
 
     // ---------------------------------------------------------------- stream and contract
     for (int ub = first_ub; active && ub < Uc; ub += shared_blocks ? Uc : W * RB) {
         const int nr = min(RB, Uc - ub);
-        if (ub != first_ub) prologue(ub, nr, pf);
+        if (ub != first_ub) prologue(ub, nr);
         uint32_t cslot = ring;
         float R[kSmMaxRB][NT][4];
 #pragma unroll
@@ -239,76 +253,76 @@ smallm_kernel(const SmallMArgs a) {
 #pragma unroll
             for (int t = 0; t < NT; ++t) R[r][t][0] = R[r][t][1] = R[r][t][2] = R[r][t][3] = 0.0f;
         for (int gl = gs0; gl < gs1; ++gl) {
-            // x fragment of the group: token 8t + g, words [16c, 16c + 16) of its 64
-            uint32_t X[NT][16];
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                const uint8_t *xp = smem + (uint32_t)(8 * t + g_l) * a.x_stride + (uint32_t)gl * 256u + c_l * 64;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(xp + 16 * q);
-                    X[t][4 * q] = v.x; X[t][4 * q + 1] = v.y; X[t][4 * q + 2] = v.z; X[t][4 * q + 3] = v.w;
-                }
+            if (pf_gl < gs1) {
+                issue(n_base + ub * 16, nr, g0 + pf_gl, pf_slot);
+                pf_slot = slot_next(pf_slot);
+                ++pf_gl;
+            } else {
+                cp_async_commit();
             }
-            // (128 + 2^(b-1)) * sum_k x[token][k] over the group, for every token column of the
-            // D fragment: the same MMA steps with a constant A operand
+            cp_async_wait_dyn(a.D - 1);
+            __syncwarp();
+            // x fragment of the group: token 8t + g, words [16c, 16c + 16) of its 64 (zeros for
+            // tokens past M); the correction (128 + 2^(b-1)) sum_k x for the fragment's columns
+            uint32_t X[NT][16];
             float corr[NT][4];
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-                corr[t][0] = corr[t][1] = corr[t][2] = corr[t][3] = 0.0f;
+                const int tok = 8 * t + g_l;
+                const uint8_t *xp = smem + (uint32_t)tok * a.x_stride + (uint32_t)gl * 256u + c_l * 64;
 #pragma unroll
-                for (int s8 = 0; s8 < 8; ++s8)
-                    mma_16816_bf16(corr[t], kBias2, kBias2, kBias2, kBias2, X[t][2 * s8], X[t][2 * s8 + 1]);
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 v = tok < M ? *reinterpret_cast<const uint4 *>(xp + 16 * q) : make_uint4(0, 0, 0, 0);
+                    X[t][4 * q] = v.x; X[t][4 * q + 1] = v.y; X[t][4 * q + 2] = v.z; X[t][4 * q + 3] = v.w;
+                }
+                const int c0 = 8 * t + 2 * c_l;
+                const float s0 = c0 < M ? sx[c0 * a.gmax + gl] : 0.0f;
+                const float s1 = c0 + 1 < M ? sx[(c0 + 1) * a.gmax + gl] : 0.0f;
+                corr[t][0] = corr[t][2] = kBiasF * s0;
+                corr[t][1] = corr[t][3] = kBiasF * s1;
             }
+            const uint8_t *slot = smem + (cslot - smem_u32(smem));
 #pragma unroll
             for (int r = 0; r < kSmMaxRB; ++r) {
-                if (r >= nr) break;
-                if (pf.gl < gs1) {
-                    issue((u0 + ub + pf.r) * 16, g0 + pf.gl, pf.slot);
-                    advance(pf, nr);
-                }
-                cp_async_commit();
-                cp_async_wait_dyn(a.D - 1);
-                __syncwarp();
-                const uint8_t *slot = smem + (cslot - smem_u32(smem));
-                cslot += a.slot_bytes;
-                if (cslot == ring + (uint32_t)a.D * a.slot_bytes) cslot = ring;
-                uint32_t wa[BITS + 1], wb[BITS + 1];
-                lds_slice<BITS>(slot + (uint32_t)g_l * kGB + c_l * 4 * BITS, wa);
-                lds_slice<BITS>(slot + (uint32_t)(g_l + 8) * kGB + c_l * 4 * BITS, wb);
-                const float sa = reinterpret_cast<const float *>(slot + 16 * kGB)[g_l];
-                const float sb = reinterpret_cast<const float *>(slot + 16 * kGB)[g_l + 8];
-                float acc[NT][CH][4];
+                if (r < nr) {
+                    uint32_t wa[BITS + 1], wb[BITS + 1];
+                    lds_slice<BITS>(slot + (uint32_t)(16 * r + g_l) * kGB + c_l * 4 * BITS, wa);
+                    lds_slice<BITS>(slot + (uint32_t)(16 * r + g_l + 8) * kGB + c_l * 4 * BITS, wb);
+                    const int row = (ub + r) * 16 + g_l;
+                    const float sa = st[row * a.gmax + gl], sb = st[(row + 8) * a.gmax + gl];
+                    float acc[NT][CH][4];
 #pragma unroll
-                for (int t = 0; t < NT; ++t)
+                    for (int t = 0; t < NT; ++t)
 #pragma unroll
-                    for (int h = 0; h < CH; ++h) acc[t][h][0] = acc[t][h][1] = acc[t][h][2] = acc[t][h][3] = 0.0f;
-                static_for<4>([&](auto bb) {
-                    constexpr int blk = decltype(bb)::value;
-                    uint32_t pa[4], pb[4];
-                    unpack_pairs_biased<BITS, blk, 1>(wa, pa);
-                    unpack_pairs_biased<BITS, blk, 1>(wb, pb);
+                        for (int h = 0; h < CH; ++h) acc[t][h][0] = acc[t][h][1] = acc[t][h][2] = acc[t][h][3] = 0.0f;
+                    static_for<4>([&](auto bb) {
+                        constexpr int blk = decltype(bb)::value;
+                        uint32_t pa[4], pb[4];
+                        unpack_pairs_biased<BITS, blk, 1>(wa, pa);
+                        unpack_pairs_biased<BITS, blk, 1>(wb, pb);
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int s8 = 2 * blk + h;
+                        for (int h = 0; h < 2; ++h) {
+                            const int s8 = 2 * blk + h;
 #pragma unroll
-                        for (int t = 0; t < NT; ++t)
-                            mma_16816_bf16(acc[t][s8 % CH], pa[2 * h], pb[2 * h], pa[2 * h + 1], pb[2 * h + 1],
-                                           X[t][2 * s8], X[t][2 * s8 + 1]);
-                    }
-                });
+                            for (int t = 0; t < NT; ++t)
+                                mma_16816_bf16(acc[t][s8 % CH], pa[2 * h], pb[2 * h], pa[2 * h + 1], pb[2 * h + 1],
+                                               X[t][2 * s8], X[t][2 * s8 + 1]);
+                        }
+                    });
 #pragma unroll
-                for (int t = 0; t < NT; ++t) {
+                    for (int t = 0; t < NT; ++t) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        float sum = acc[t][0][k] - corr[t][k];
+                        for (int k = 0; k < 4; ++k) {
+                            float sum = acc[t][0][k] - corr[t][k];
 #pragma unroll
-                        for (int h = 1; h < CH; ++h) sum += acc[t][h][k];
-                        R[r][t][k] = fmaf(k < 2 ? sa : sb, sum, R[r][t][k]);
+                            for (int h = 1; h < CH; ++h) sum += acc[t][h][k];
+                            R[r][t][k] = fmaf(k < 2 ? sa : sb, sum, R[r][t][k]);
+                        }
                     }
                 }
-                __syncwarp();          // every lane is done with the slot before it is refilled
             }
+            __syncwarp();              // every lane is done with the slot before it is refilled
+            cslot = slot_next(cslot);
         }
         // this block's partial sums -> part[split][token][row of the cluster range]
         float *ps = part + split * part_stride;
@@ -329,7 +343,7 @@ smallm_kernel(const SmallMArgs a) {
     __syncthreads();
     // ---------------------------------------------------------------- CTA reduction (fixed order)
     if (shared_blocks && a.GW > 1) {
-        for (int e = threadIdx.x; e < TOK * rows_c; e += W * 32) {
+        for (int e = threadIdx.x; e < M * rows_c; e += W * 32) {
             const int tok = e / rows_c, row = e - tok * rows_c;
             float v = part[tok * a.rows_max + row];
             for (int j = 1; j < a.GW; ++j) v += part[j * part_stride + tok * a.rows_max + row];
@@ -339,9 +353,8 @@ smallm_kernel(const SmallMArgs a) {
     }
     if (S > 1) cluster_sync();
     // ---------------------------------------------------------------- finalize a 1/S share
-    const int64_t n_base = u0 * 16;
     const int rows_v = (int)min((int64_t)rows_c, a.N - n_base);
-    const int E = (int)a.M * rows_v;
+    const int E = M * rows_v;
     const int e0 = (int)((int64_t)E * srank / S), e1 = (int)((int64_t)E * (srank + 1) / S);
     const uint32_t part_addr = smem_u32(part);
     for (int e = e0 + (int)threadIdx.x; e < e1; e += W * 32) {

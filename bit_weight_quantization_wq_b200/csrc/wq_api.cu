@@ -215,21 +215,24 @@ int small_max_clusters(int dev, int S, int sm_count) {
 // each warp streams its items through D ring slots. Returns the busiest warp's item count,
 // or -1 when nothing fits in shared memory.
 template <int BITS, int TOK>
-int64_t small_plan(int64_t U, int G, int S, int C, wq::SmallMArgs &a, uint32_t *smem_total) {
+int64_t small_plan(int64_t U, int G, int S, int C, int M, wq::SmallMArgs &a, uint32_t *smem_total) {
     constexpr int W = wq::SmCfg<TOK>::kWarps;
     const int64_t uc = (U + C - 1) / C;
     const int gc = (G + S - 1) / S;
     const uint32_t x_stride = (uint32_t)gc * 256u + 64u;
-    const uint32_t x_bytes = align_u32((uint32_t)TOK * x_stride, 128);
-    const uint32_t slot = 16u * 16u * BITS + 64u;
+    const uint32_t x_bytes = align_u32((uint32_t)M * x_stride, 128);
+    const uint32_t sx_bytes = align_u32((uint32_t)TOK * (uint32_t)gc * 4u, 128);
+    const uint32_t st_bytes = align_u32((uint32_t)(uc * 16) * (uint32_t)gc * 4u, 128);
+    const uint32_t fixed = x_bytes + sx_bytes + st_bytes;
     int64_t best = -1;
     for (int rb = wq::kSmMaxRB; rb >= 1; --rb) {
         const int64_t nb = (uc + rb - 1) / rb;
         const int gw = nb >= W ? 1 : (int)(W / nb);
         const int64_t items = nb >= W ? ((nb + W - 1) / W) * rb * gc : (int64_t)rb * ((gc + gw - 1) / gw);
         const uint32_t part = align_u32((uint32_t)gw * TOK * (uint32_t)(uc * 16) * 4u, 128);
+        const uint32_t slot = (uint32_t)rb * 16u * 16u * BITS;
         for (int d = wq::kSmMaxD; d >= 2; --d) {
-            const uint32_t total = x_bytes + (uint32_t)W * d * slot + part;
+            const uint32_t total = fixed + (uint32_t)W * d * slot + part;
             if (total > kSmemMax) continue;
             // fewer items per warp first; then a deeper ring, then more x reuse (larger blocks)
             const int64_t cost = items * 8 + (d >= 4 ? 0 : 4 - d);
@@ -239,10 +242,13 @@ int64_t small_plan(int64_t U, int G, int S, int C, wq::SmallMArgs &a, uint32_t *
                 a.GW = gw;
                 a.D = d;
                 a.rows_max = (int)(uc * 16);
+                a.gmax = gc;
                 a.x_stride = x_stride;
                 a.slot_bytes = slot;
-                a.off_ring = x_bytes;
-                a.off_part = x_bytes + (uint32_t)W * d * slot;
+                a.off_sx = x_bytes;
+                a.off_st = x_bytes + sx_bytes;
+                a.off_ring = fixed;
+                a.off_part = fixed + (uint32_t)W * d * slot;
                 *smem_total = total;
             }
             break;
@@ -273,7 +279,7 @@ wq_status launch_smallm_tok(wq::SmallMArgs a, int dev, int sm_count, cudaStream_
         const int C = (int)std::min<int64_t>(mc, U);
         wq::SmallMArgs t = a;
         uint32_t total = 0;
-        const int64_t cost = small_plan<BITS, TOK>(U, G, S, C, t, &total);
+        const int64_t cost = small_plan<BITS, TOK>(U, G, S, C, (int)a.M, t, &total);
         if (cost < 0) continue;
         if (best < 0 || cost < best) {
             best = cost;
@@ -419,23 +425,29 @@ template <int R>
 wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_t st) {
     const int64_t mtiles = (a.M + 63) / 64;
     const int64_t nkb = a.K / 64;
-    // The prepass is latency-bound (each CTA walks its K share one 64-k block at a time), so
-    // K is split (clusters of up to 16 CTAs, a non-portable size) until about eight CTAs per
-    // SM are in flight.
+    // K is split over a cluster of up to 16 CTAs (a non-portable size) while that leaves fewer
+    // than two CTAs per SM; each CTA stages its share of L1 in shared memory, in passes of sb
+    // 64-k blocks (a multiple of the x prefetch depth) when it does not fit at once
+    int ks = 1;
+    while (ks < wq::kPreMaxKS && ks * 2 <= nkb && mtiles * ks < 2 * (int64_t)sm_count) ks *= 2;
+    const int nb_max = (int)((nkb + ks - 1) / ks);
+    int sb = (nb_max + wq::kPrePf - 1) / wq::kPrePf * wq::kPrePf;
+    while (sb > wq::kPrePf && wq::prepass_smem_bytes<R>(sb) > kSmemMax / 2) sb -= wq::kPrePf;   // two CTAs per SM
+    const uint32_t smem = wq::prepass_smem_bytes<R>(sb);
     static std::atomic<int> attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     cudaError_t e = setup_once(attr_done, dev, [] {
-        return cudaFuncSetAttribute(wq::lowrank_prepass_kernel<R>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        cudaError_t r = cudaFuncSetAttribute(wq::lowrank_prepass_kernel<R>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (r != cudaSuccess) return r;
+        return cudaFuncSetAttribute(wq::lowrank_prepass_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSmemMax);
     });
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(lowrank_prepass_kernel)");
-    const int kmax = 16;
-    int ks = 1;
-    while (ks < kmax && ks * 2 <= nkb && mtiles * ks < 8 * (int64_t)sm_count) ks *= 2;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)mtiles, (unsigned)ks, 1);
     cfg.blockDim = dim3(128);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -445,7 +457,7 @@ wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, wq::lowrank_prepass_kernel<R>, static_cast<const uint16_t *>(a.x),
-                                       static_cast<const uint16_t *>(a.L1), t, a.M, a.K);
+                           static_cast<const uint16_t *>(a.L1), t, a.M, a.K, sb);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(lowrank_prepass_kernel)");
     return check_launch("lowrank_prepass_kernel");
 }
