@@ -313,6 +313,16 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
     return v;
 }
 
+// ------------------------------------------------------------------ dependent launches
+// A kernel launched with programmatic stream serialization may start while the launch before
+// it on the stream is still running; it waits here, before it reads anything that launch
+// writes, until that launch has completed and its writes are visible. Without the launch
+// attribute the wait returns at once.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next launch on the stream start early (it still waits for this one in
+// grid_dependency_wait before reading what this one writes).
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ misc
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h16) {
     return __uint_as_float(h16 << 16);

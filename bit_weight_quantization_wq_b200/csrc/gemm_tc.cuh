@@ -501,6 +501,7 @@ lowrank_prepass_kernel(const uint16_t *__restrict__ x, const uint16_t *__restric
     uint16_t *l1s = reinterpret_cast<uint16_t *>(pre_smem);                   // [sb*64][kLd]
     float *part = reinterpret_cast<float *>(pre_smem + (size_t)sb * 64 * kLd * 2); // [64][R]
     const int64_t ra = m0 + warp * 16 + g, rb = ra + 8;
+    grid_launch_dependents();                           // the consumer of t waits for this grid's end
 
     // blocks [b0, b1) of this CTA's share of L1 -> shared memory (asynchronous 16-byte copies)
     auto stage_l1 = [&](int b0, int b1) {

@@ -19,8 +19,10 @@
 // private ring of D slots in shared memory, D - 1 groups ahead of the one being computed;
 // the warp waits on its own copy groups only. There is no producer warp and no barrier
 // between warps until the final reduction. At the start the CTA copies into shared memory,
-// once: the token rows of x for its groups (padded stride), every group's sum of x per
-// token, and the steps of all its rows and groups.
+// once, with asynchronous copies that are in flight together with the ring's first slots:
+// the token rows of x for its groups (padded stride), the steps of all its rows and groups
+// and, with a low-rank branch, the L2 columns of its rows; then it sums every staged group of
+// x per token.
 //
 // Arithmetic: thread (g, c) of a warp holds rows g and g+8 of the unit and the 32
 // consecutive codes [32c, 32c+32) of the group, 4*b contiguous bytes per row. Inside one
@@ -34,7 +36,10 @@
 //
 // Reduction: warps that share a block add their partial sums in a fixed order through
 // shared memory, then the S CTAs of a cluster add theirs through distributed shared memory
-// (in rank order), add the low-rank branch and the bias, and round once to bf16. All orders
+// (in rank order), add the low-rank branch and the bias, and round once to bf16. The
+// low-rank input t = x L1 is written by a prepass launched just before this kernel; this
+// kernel is launched as its programmatic dependent, streams the weight while the prepass
+// runs, and waits for it only before the finish. All orders
 // are fixed: the result is deterministic. The kernel has no waits on other threads' progress
 // except __syncthreads and the cluster barrier, which every thread reaches.
 #pragma once
@@ -78,6 +83,8 @@ struct SmallMArgs {
     uint32_t x_stride;        // bytes per token row of the staged x (gmax * 256 + 64)
     uint32_t slot_bytes;      // one ring slot: RB units x 16 rows x 16b bytes of codes
     uint32_t off_sx, off_st, off_ring, off_part;
+    uint32_t off_l2;          // staged L2 columns of the cluster's rows, [rank][rows_max] bf16
+    int l2_staged;            // 1 when L2 is staged (rows of 16-byte multiples: N % 8 == 0)
 };
 
 // ---------------------------------------------------------------- asynchronous copies
@@ -192,7 +199,39 @@ smallm_kernel(const SmallMArgs a) {
     };
     auto slot_next = [&](uint32_t s) { s += a.slot_bytes; return s == ring + (uint32_t)a.D * a.slot_bytes ? ring : s; };
 
-    // first copies go out before the staging, so the ring fills while x arrives
+    // ---------------------------------------------------------------- stage x, steps
+    // One commit group of asynchronous copies, issued before the ring prologue so that both
+    // are in flight together: the token rows of x for the CTA's groups and the steps of its
+    // rows and groups.
+    {
+        const int chunks = Gc * 16;                            // 16-byte chunks per token row
+        const uint32_t xs = smem_u32(smem);
+        for (int e = threadIdx.x; e < M * chunks; e += W * 32) {
+            const int tok = e / chunks, j = e - tok * chunks;
+            cp_async_16(xs + (uint32_t)tok * a.x_stride + 16u * j, a.x + (int64_t)tok * a.K + (int64_t)g0 * 128 + 8 * j, 16u);
+        }
+        const int rows_v = (int)min((int64_t)rows_c, a.N - n_base);
+        const uint32_t ss = smem_u32(st);
+        for (int e = threadIdx.x; e < rows_v * Gc; e += W * 32) {
+            const int i = e / Gc, gl = e - i * Gc;
+            cp_async_4(ss + 4u * (uint32_t)(i * a.gmax + gl), a.scales + (n_base + i) * G + g0 + gl, 4u);
+        }
+        if (a.l2_staged) {
+            // L2 columns [n_base, n_base + rows_c) of every rank row, 8 columns per copy (zeros past N)
+            const int per_row = rows_c / 8;
+            const uint32_t ls = smem_u32(smem + a.off_l2);
+            for (int e = threadIdx.x; e < a.rank * per_row; e += W * 32) {
+                const int jr = e / per_row, cj = e - jr * per_row;
+                const int64_t n = n_base + 8 * cj;
+                const bool ok = n < a.N;
+                cp_async_16(ls + 2u * (uint32_t)(jr * a.rows_max + 8 * cj), ok ? a.L2 + (int64_t)jr * a.N + n : a.L2,
+                            ok ? 16u : 0u);
+            }
+        }
+        cp_async_commit();
+    }
+
+    // the ring's first D - 1 slots, also in flight while the staging copies land
     const int first_ub = shared_blocks ? (warp % NB) * RB : warp * RB;
     uint32_t pf_slot = ring;
     int pf_gl = gs0;
@@ -209,36 +248,35 @@ smallm_kernel(const SmallMArgs a) {
             }
         }
     };
-    if (active && first_ub < Uc) prologue(first_ub, min(RB, Uc - first_ub));
-
-    // ---------------------------------------------------------------- stage x, steps
-    {
-        const int chunks = Gc * 16;                            // 16-byte chunks per token row
-        for (int e = threadIdx.x; e < M * chunks; e += W * 32) {
-            const int tok = e / chunks, j = e - tok * chunks;
-            const uint4 v = ldg_stream_v4(a.x + (int64_t)tok * a.K + (int64_t)g0 * 128 + 8 * j);
-            *reinterpret_cast<uint4 *>(smem + (uint32_t)tok * a.x_stride + 16u * j) = v;
-        }
-        const int rows_v = (int)min((int64_t)rows_c, a.N - n_base);
-        for (int e = threadIdx.x; e < rows_v * Gc; e += W * 32) {
-            const int i = e / Gc, gl = e - i * Gc;
-            st[i * a.gmax + gl] = __ldg(a.scales + (n_base + i) * G + g0 + gl);
-        }
+    if (active && first_ub < Uc) {
+        prologue(first_ub, min(RB, Uc - first_ub));
+        cp_async_wait_dyn(a.D - 1);                            // the staging group is the oldest
+    } else {
+        cp_async_wait<0>();
     }
     __syncthreads();
-    // sum of each staged token row over each group (fixed order)
-    for (int e = threadIdx.x; e < M * Gc; e += W * 32) {
-        const int tok = e / Gc, gl = e - tok * Gc;
-        const uint4 *xp = reinterpret_cast<const uint4 *>(smem + (uint32_t)tok * a.x_stride + (uint32_t)gl * 256u);
+    // sum of each staged token row over each group: 8 lanes per (token, group), 16 values
+    // each, then a fixed xor tree over the 8 lanes (deterministic)
+    for (int base = warp * 32; base < M * Gc * 8; base += W * 32) {
+        const int e = base + lane;
+        const bool ok = e < M * Gc * 8;
+        const int item = e >> 3, part8 = e & 7;
+        const int tok = ok ? item / Gc : 0, gl = ok ? item - tok * Gc : 0;
         float sum = 0.0f;
-#pragma unroll 4
-        for (int q = 0; q < 16; ++q) {
-            const uint4 v = xp[q];
-            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        if (ok) {
+            const uint4 *xp = reinterpret_cast<const uint4 *>(smem + (uint32_t)tok * a.x_stride + (uint32_t)gl * 256u +
+                                                              32u * part8);
+            const uint4 v0 = xp[0], v1 = xp[1];
+            const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            float h[8];
 #pragma unroll
-            for (int h = 0; h < 4; ++h) sum += bf16_bits_to_f32(wv[h] & 0xFFFFu) + bf16_bits_to_f32(wv[h] >> 16);
+            for (int q = 0; q < 8; ++q) h[q] = bf16_bits_to_f32(wv[q] & 0xFFFFu) + bf16_bits_to_f32(wv[q] >> 16);
+            sum = ((h[0] + h[1]) + (h[2] + h[3])) + ((h[4] + h[5]) + (h[6] + h[7]));
         }
-        sx[tok * a.gmax + gl] = sum;
+        sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        if (ok && part8 == 0) sx[tok * a.gmax + gl] = sum;
     }
     __syncthreads();
 
@@ -352,32 +390,70 @@ smallm_kernel(const SmallMArgs a) {
         __syncthreads();
     }
     if (S > 1) cluster_sync();
+    // ---------------------------------------------------------------- low-rank input
+    // t = x L1 comes from the launch before this one, which may still be running: wait for
+    // it, then hold t_hi + t_lo per token and rank column in fp32 where the ring was
+    float *ts = reinterpret_cast<float *>(smem + a.off_ring);
+    if (a.rank > 0) {
+        grid_dependency_wait();
+        for (int e = threadIdx.x; e < M * a.rank; e += W * 32) {
+            const int m = e / a.rank, jr = e - m * a.rank;
+            const uint16_t *tm = a.t + (int64_t)m * kTStrideSm;
+            ts[e] = bf16_bits_to_f32(tm[jr]) + bf16_bits_to_f32(tm[a.rank + jr]);
+        }
+        __syncthreads();
+    }
     // ---------------------------------------------------------------- finalize a 1/S share
+    // Each thread finishes kFin outputs at a time so that their partial-sum loads overlap.
+    constexpr int kFin = 4;
     const int rows_v = (int)min((int64_t)rows_c, a.N - n_base);
     const int E = M * rows_v;
     const int e0 = (int)((int64_t)E * srank / S), e1 = (int)((int64_t)E * (srank + 1) / S);
     const uint32_t part_addr = smem_u32(part);
-    for (int e = e0 + (int)threadIdx.x; e < e1; e += W * 32) {
-        const int m = e / rows_v, i = e - m * rows_v;
-        const uint32_t off = 4u * (uint32_t)(m * a.rows_max + i);
-        float v = 0.0f;
+    const uint16_t *l2s = reinterpret_cast<const uint16_t *>(smem + a.off_l2);
+    for (int eb = e0 + (int)threadIdx.x; eb < e1; eb += kFin * W * 32) {
+        float v[kFin];
+        int mm[kFin], ii[kFin];
+#pragma unroll
+        for (int u = 0; u < kFin; ++u) {
+            const int e = eb + u * W * 32;
+            mm[u] = e < e1 ? e / rows_v : 0;
+            ii[u] = e < e1 ? e - mm[u] * rows_v : 0;
+            v[u] = 0.0f;
+        }
         if (S > 1) {
-            for (int q = 0; q < S; ++q) v += ld_cluster_f32(map_cluster_smem(part_addr + off, (uint32_t)q));
-        } else {
-            v = part[m * a.rows_max + i];
-        }
-        const int64_t n = n_base + i;
-        if (a.rank > 0) {
-            const uint16_t *tm = a.t + (int64_t)m * kTStrideSm;
-            float lr = 0.0f;
-            for (int jr = 0; jr < a.rank; ++jr) {
-                const float tv = bf16_bits_to_f32(tm[jr]) + bf16_bits_to_f32(tm[a.rank + jr]);
-                lr = fmaf(tv, bf16_bits_to_f32(__ldg(a.L2 + (int64_t)jr * a.N + n)), lr);
+            for (int q = 0; q < S; ++q) {
+#pragma unroll
+                for (int u = 0; u < kFin; ++u)
+                    if (eb + u * W * 32 < e1)
+                        v[u] += ld_cluster_f32(map_cluster_smem(part_addr + 4u * (uint32_t)(mm[u] * a.rows_max + ii[u]),
+                                                                (uint32_t)q));
             }
-            v += lr;
+        } else {
+#pragma unroll
+            for (int u = 0; u < kFin; ++u)
+                if (eb + u * W * 32 < e1) v[u] = part[mm[u] * a.rows_max + ii[u]];
         }
-        if (a.bias) v += bf16_bits_to_f32(__ldg(a.bias + n));
-        a.y[(int64_t)m * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+#pragma unroll
+        for (int u = 0; u < kFin; ++u) {
+            if (eb + u * W * 32 >= e1) break;
+            const int64_t n = n_base + ii[u];
+            float acc = v[u];
+            if (a.rank > 0) {
+                const float *tm = ts + mm[u] * a.rank;
+                float lr = 0.0f;
+                if (a.l2_staged) {
+                    for (int jr = 0; jr < a.rank; ++jr)
+                        lr = fmaf(tm[jr], bf16_bits_to_f32(l2s[jr * a.rows_max + ii[u]]), lr);
+                } else {
+                    for (int jr = 0; jr < a.rank; ++jr)
+                        lr = fmaf(tm[jr], bf16_bits_to_f32(__ldg(a.L2 + (int64_t)jr * a.N + n)), lr);
+                }
+                acc += lr;
+            }
+            if (a.bias) acc += bf16_bits_to_f32(__ldg(a.bias + n));
+            a.y[(int64_t)mm[u] * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+        }
     }
     if (S > 1) cluster_sync();       // no CTA leaves while another may still read its part[]
 }

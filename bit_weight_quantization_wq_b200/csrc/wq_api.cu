@@ -223,7 +223,10 @@ int64_t small_plan(int64_t U, int G, int S, int C, int M, wq::SmallMArgs &a, uin
     const uint32_t x_bytes = align_u32((uint32_t)M * x_stride, 128);
     const uint32_t sx_bytes = align_u32((uint32_t)TOK * (uint32_t)gc * 4u, 128);
     const uint32_t st_bytes = align_u32((uint32_t)(uc * 16) * (uint32_t)gc * 4u, 128);
-    const uint32_t fixed = x_bytes + sx_bytes + st_bytes;
+    // L2 columns of the cluster's rows, staged when its rows are 16-byte multiples
+    const bool l2_staged = a.rank > 0 && a.N % 8 == 0;
+    const uint32_t l2_bytes = l2_staged ? align_u32((uint32_t)a.rank * (uint32_t)(uc * 16) * 2u, 128) : 0u;
+    const uint32_t fixed = x_bytes + sx_bytes + st_bytes + l2_bytes;
     int64_t best = -1;
     for (int rb = wq::kSmMaxRB; rb >= 1; --rb) {
         const int64_t nb = (uc + rb - 1) / rb;
@@ -247,6 +250,8 @@ int64_t small_plan(int64_t U, int G, int S, int C, int M, wq::SmallMArgs &a, uin
                 a.slot_bytes = slot;
                 a.off_sx = x_bytes;
                 a.off_st = x_bytes + sx_bytes;
+                a.off_l2 = x_bytes + sx_bytes + st_bytes;
+                a.l2_staged = l2_staged ? 1 : 0;
                 a.off_ring = fixed;
                 a.off_part = fixed + (uint32_t)W * d * slot;
                 *smem_total = total;
@@ -295,13 +300,24 @@ wq_status launch_smallm_tok(wq::SmallMArgs a, int dev, int sm_count, cudaStream_
     cfg.blockDim = dim3(wq::SmCfg<TOK>::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)chosen.S;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    unsigned n_attr = 0;
+    if (chosen.S > 1) {
+        attr[n_attr].id = cudaLaunchAttributeClusterDimension;
+        attr[n_attr].val.clusterDim.x = (unsigned)chosen.S;
+        attr[n_attr].val.clusterDim.y = 1;
+        attr[n_attr].val.clusterDim.z = 1;
+        ++n_attr;
+    }
+    if (chosen.rank > 0) {
+        // t comes from the prepass launched just before: the kernel streams the weight while
+        // the prepass runs and waits for it (griddepcontrol.wait) only before reading t
+        attr[n_attr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n_attr].val.programmaticStreamSerializationAllowed = 1;
+        ++n_attr;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = chosen.S > 1 ? 1 : 0;
+    cfg.numAttrs = n_attr;
     e = cudaLaunchKernelEx(&cfg, wq::smallm_kernel<BITS, TOK>, chosen);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(smallm_kernel)");
     return check_launch("smallm_kernel");
