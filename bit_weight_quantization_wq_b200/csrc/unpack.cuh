@@ -105,25 +105,49 @@ __device__ __forceinline__ void unpack_pairs(const uint32_t (&w)[NW], uint32_t (
 
 // As unpack_pairs, but each half is the bf16 value 128 + code (no subtraction): the caller
 // removes (128 + 2^(b-1)) * sum(x) once per group instead of once per code pair.
-// 4 bits: byte j of a word = (code 2j << 4) | code 2j+1; two permutes interleave the high
-// and low nibbles into code order, then one permute per pair pairs two code bytes with the
-// constant byte 0x43 (bf16 0x43cc = 128 + c for c < 16).
+//
+// 4 bits: the pairs come out in a permuted k order. Byte j of a block word is
+// (code 2j << 4) | code 2j+1, so one mask keeps one nibble of each 16-bit half: bits [0,4)
+// and [16,20) hold codes 1 and 5, and shifts by 4, 8 and 12 bring codes (0,4), (3,7) and
+// (2,6) there. Word i of the block's output holds the pair (i, i+4), which is exact bf16
+// 128 + code with the constant 0x4300 in each half: three shifts and four mask-and-or
+// operations per 8 codes. The x operand of the MMA then takes the same order: see
+// permute_x8. Other widths return pairs in natural order (word i = codes 2i, 2i+1).
+template <int BITS> struct BiasedOrder { static constexpr bool kPermuted = (BITS == 4); };
+
+// (a & b) | c in one instruction; b and c are registers, so the two constants of the biased
+// unpack do not become two immediates of two instructions.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// The two constants of the biased unpack for width BITS, held in registers: the per-half
+// code mask and the bf16 exponent pattern 0x4300 in each half.
+template <int BITS> struct BiasedConsts {
+    uint32_t mask, one;
+    __device__ __forceinline__ BiasedConsts() {
+        constexpr uint32_t m = (1u << (BITS == 4 ? 4 : BITS)) - 1u;
+        mask = m | (m << 16);
+        one = 0x43004300u;
+        asm volatile("" : "+r"(mask), "+r"(one));       // keep them in registers
+    }
+};
+
 template <int BITS, int BLK0, int NBLK, int NW>
-__device__ __forceinline__ void unpack_pairs_biased(const uint32_t (&w)[NW], uint32_t (&out)[4 * NBLK]) {
+__device__ __forceinline__ void unpack_pairs_biased(const uint32_t (&w)[NW], uint32_t (&out)[4 * NBLK],
+                                                    const BiasedConsts<BITS> &k) {
     if constexpr (BITS == 4) {
 #pragma unroll
         for (int i = 0; i < NBLK; ++i) {
             const uint32_t v = w[BLK0 + i];
-            const uint32_t hiN = (v >> 4) & 0x0F0F0F0Fu, loN = v & 0x0F0F0F0Fu;
-            const uint32_t c03 = __byte_perm(hiN, loN, 0x5140u);     // codes 0..3 as bytes
-            const uint32_t c47 = __byte_perm(hiN, loN, 0x7362u);     // codes 4..7
-            out[4 * i + 0] = __byte_perm(c03, 0x43434343u, 0x4140u);
-            out[4 * i + 1] = __byte_perm(c03, 0x43434343u, 0x4342u);
-            out[4 * i + 2] = __byte_perm(c47, 0x43434343u, 0x4140u);
-            out[4 * i + 3] = __byte_perm(c47, 0x43434343u, 0x4342u);
+            out[4 * i + 0] = and_or(v >> 4, k.mask, k.one);     // codes 0, 4
+            out[4 * i + 1] = and_or(v, k.mask, k.one);          // codes 1, 5
+            out[4 * i + 2] = and_or(v >> 12, k.mask, k.one);    // codes 2, 6
+            out[4 * i + 3] = and_or(v >> 8, k.mask, k.one);     // codes 3, 7
         }
     } else {
-        constexpr uint32_t m = (1u << BITS) - 1u;
         static_for<NBLK>([&](auto bb) {
             constexpr int blk = decltype(bb)::value;
             uint32_t lo, hi;
@@ -135,10 +159,17 @@ __device__ __forceinline__ void unpack_pairs_biased(const uint32_t (&w)[NW], uin
                 if constexpr (sh >= 32) G = hi >> (sh - 32);
                 else if constexpr (sh == 0) G = lo;
                 else G = __funnelshift_r(lo, hi, sh);
-                out[4 * blk + pr] = (__byte_perm(G >> BITS, G, 0x5410u) & (m | (m << 16))) | 0x43004300u;
+                out[4 * blk + pr] = and_or(__byte_perm(G >> BITS, G, 0x5410u), k.mask, k.one);
             });
         });
     }
+}
+
+// Eight bf16 values x0..x7 (four words, natural order) -> the order the 4-bit biased pairs
+// take: words (x0, x4), (x1, x5), (x2, x6), (x3, x7).
+__device__ __forceinline__ uint4 permute_x8(const uint4 v) {
+    return make_uint4(__byte_perm(v.x, v.z, 0x5410u), __byte_perm(v.x, v.z, 0x7632u),
+                      __byte_perm(v.y, v.w, 0x5410u), __byte_perm(v.y, v.w, 0x7632u));
 }
 
 // mma.m16n8k16, bf16 inputs, fp32 accumulate in place.

@@ -176,7 +176,10 @@ wq_status launch_error_many(const wq_error_job *jobs, int n_jobs, int sm_count, 
 // ------------------------------------------------------------------ small-M path
 constexpr uint32_t kSmemMax = 227 * 1024;        // dynamic shared memory per CTA on sm_100
 
-uint32_t align_u32(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+uint64_t align_u64(uint64_t v, uint64_t a) { return (v + a - 1) / a * a; }
+
+wq_status make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
 
 // Clusters of S CTAs that fit at once (one CTA per SM, the most shared memory), cached.
 template <int BITS, int TOK>
@@ -200,7 +203,7 @@ int small_max_clusters(int dev, int S, int sm_count) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int q = 0;
-        if (cudaOccupancyMaxActiveClusters(&q, (void *)wq::smallm_kernel<BITS, TOK>, &cfg) != cudaSuccess) q = 0;
+        if (cudaOccupancyMaxActiveClusters(&q, (void *)wq::smallm_kernel<BITS, TOK, 1>, &cfg) != cudaSuccess) q = 0;
         cudaGetLastError();
         n = std::min(n, q);
     }
@@ -212,62 +215,92 @@ int small_max_clusters(int dev, int S, int sm_count) {
 // Work split and shared-memory layout of smallm_kernel for a cluster size S: C clusters own
 // ~U/C units each, a CTA ~G/S groups. Inside the CTA, blocks of RB units go to the W warps
 // (GW warps per block, each a share of the groups, when there are fewer blocks than warps);
-// each warp streams its items through D ring slots. Returns the busiest warp's item count,
-// or -1 when nothing fits in shared memory.
+// each warp streams its items through D ring slots. Returns the busiest warp's item count
+// (scaled, with a small preference for deeper rings), or -1 when nothing fits.
+//
+// Layout: x [M][x_stride] | 256 zero bytes at 64 mod 128 | st [gc][rows_pad] | L2 [rank][rows_max] |
+// mbarriers [W][D], staging mbarrier, abort word | rings [W][D][slot] | part [GW][TOK][rows_max].
 template <int BITS, int TOK>
 int64_t small_plan(int64_t U, int G, int S, int C, int M, wq::SmallMArgs &a, uint32_t *smem_total) {
     constexpr int W = wq::SmCfg<TOK>::kWarps;
     const int64_t uc = (U + C - 1) / C;
     const int gc = (G + S - 1) / S;
-    const uint32_t x_stride = (uint32_t)gc * 256u + 64u;
-    const uint32_t x_bytes = align_u32((uint32_t)M * x_stride, 128);
-    const uint32_t sx_bytes = align_u32((uint32_t)TOK * (uint32_t)gc * 4u, 128);
-    const uint32_t st_bytes = align_u32((uint32_t)(uc * 16) * (uint32_t)gc * 4u, 128);
-    // L2 columns of the cluster's rows, staged when its rows are 16-byte multiples
-    const bool l2_staged = a.rank > 0 && a.N % 8 == 0;
-    const uint32_t l2_bytes = l2_staged ? align_u32((uint32_t)a.rank * (uint32_t)(uc * 16) * 2u, 128) : 0u;
-    const uint32_t fixed = x_bytes + sx_bytes + st_bytes + l2_bytes;
+    // sizes in 64 bits: a layout is kept only when its total fits in shared memory
+    const uint64_t x_stride = (uint64_t)gc * 256u + 64u;
+    const uint64_t x_bytes = align_u64((uint64_t)M * x_stride, 128);
+    const uint64_t off_zero = x_bytes + 64u;
+    const uint64_t off_st = x_bytes + 384u;
     int64_t best = -1;
-    for (int rb = wq::kSmMaxRB; rb >= 1; --rb) {
-        const int64_t nb = (uc + rb - 1) / rb;
-        const int gw = nb >= W ? 1 : (int)(W / nb);
-        const int64_t items = nb >= W ? ((nb + W - 1) / W) * rb * gc : (int64_t)rb * ((gc + gw - 1) / gw);
-        const uint32_t part = align_u32((uint32_t)gw * TOK * (uint32_t)(uc * 16) * 4u, 128);
-        const uint32_t slot = (uint32_t)rb * 16u * 16u * BITS;
-        for (int d = wq::kSmMaxD; d >= 2; --d) {
-            const uint32_t total = fixed + (uint32_t)W * d * slot + part;
-            if (total > kSmemMax) continue;
-            // fewer items per warp first; then a deeper ring, then more x reuse (larger blocks)
-            const int64_t cost = items * 8 + (d >= 4 ? 0 : 4 - d);
-            if (best < 0 || cost < best) {
-                best = cost;
-                a.RB = rb;
-                a.GW = gw;
-                a.D = d;
-                a.rows_max = (int)(uc * 16);
-                a.gmax = gc;
-                a.x_stride = x_stride;
-                a.slot_bytes = slot;
-                a.off_sx = x_bytes;
-                a.off_st = x_bytes + sx_bytes;
-                a.off_l2 = x_bytes + sx_bytes + st_bytes;
-                a.l2_staged = l2_staged ? 1 : 0;
-                a.off_ring = fixed;
-                a.off_part = fixed + (uint32_t)W * d * slot;
-                *smem_total = total;
+    // L2 columns of the cluster's rows are staged when its rows are 16-byte multiples and the
+    // layout still fits; otherwise the finish reads them from global memory
+    for (int l2_try = 1; l2_try >= 0 && best < 0; --l2_try) {
+        const bool l2_staged = l2_try == 1 && a.rank > 0 && a.N % 8 == 0;
+        if (l2_try == 1 && !l2_staged) continue;
+        const uint64_t l2_bytes = l2_staged ? align_u64((uint64_t)a.rank * (uint64_t)(uc * 16) * 2u, 128) : 0u;
+        for (int rb = wq::sm_max_rb<TOK>(); rb >= 1; --rb) {
+            const int64_t nb = (uc + rb - 1) / rb;
+            const int gw = nb >= W ? 1 : (int)(W / nb);
+            // items (one group of one block) on the busiest warp; an item costs about one unit's
+            // work on top of its units' (the x fragment, the correction MMAs, the wait and copy)
+            const int64_t items = nb >= W ? ((nb + W - 1) / W) * gc : (gc + gw - 1) / gw;
+            const int64_t rows_pad = uc * 16 + 16 * (rb - 1);
+            const uint64_t st_bytes = align_u64((uint64_t)rows_pad * (uint64_t)gc * 4u, 128);
+            const uint64_t off_l2 = off_st + st_bytes;
+            const uint64_t off_bar = off_l2 + l2_bytes;
+            const uint64_t part = align_u64((uint64_t)gw * TOK * (uint64_t)(uc * 16) * 4u, 128);
+            const uint64_t slot = (uint64_t)rb * 16u * 16u * BITS;
+            for (int d = wq::kSmMaxD; d >= 2; --d) {
+                const uint64_t off_ring = off_bar + align_u64((uint64_t)W * d * 8u + 16u, 128);   // + staging bar, abort
+                const uint64_t total = off_ring + (uint64_t)W * d * slot + part;
+                if (total > kSmemMax) continue;
+                // the least work on the busiest warp first; then a deeper ring
+                const int64_t cost = items * (1 + rb) * 8 + (d >= 4 ? 0 : 4 - d);
+                if (best < 0 || cost < best) {
+                    best = cost;
+                    a.RB = rb;
+                    a.GW = gw;
+                    a.D = d;
+                    a.rows_max = (int)(uc * 16);
+                    a.rows_pad = (int)rows_pad;
+                    a.gmax = gc;
+                    a.x_stride = (uint32_t)x_stride;
+                    a.slot_bytes = (uint32_t)slot;
+                    a.off_zero = (uint32_t)off_zero;
+                    a.off_st = (uint32_t)off_st;
+                    a.off_l2 = (uint32_t)off_l2;
+                    a.off_bar = (uint32_t)off_bar;
+                    a.off_ring = (uint32_t)off_ring;
+                    a.off_part = (uint32_t)(off_ring + (uint64_t)W * d * slot);
+                    a.l2_staged = l2_staged ? 1 : 0;
+                    *smem_total = (uint32_t)total;
+                }
+                break;
             }
-            break;
         }
     }
     return best;
 }
 
+template <int BITS, int TOK, int RB>
+cudaError_t smallm_launch_rb(const cudaLaunchConfig_t &cfg, const CUtensorMap &pm, const wq::SmallMArgs &a) {
+    return cudaLaunchKernelEx(&cfg, wq::smallm_kernel<BITS, TOK, RB>, pm, a);
+}
+
+// *no_layout is set (and nothing launched) when no cluster size has a shared-memory layout
+// for this many tokens.
 template <int BITS, int TOK>
-wq_status launch_smallm_tok(wq::SmallMArgs a, int dev, int sm_count, cudaStream_t st) {
+wq_status launch_smallm_tok(wq::SmallMArgs a, const CUtensorMap &pm, int dev, int sm_count, cudaStream_t st,
+                            bool *no_layout) {
+    *no_layout = false;
     static std::atomic<int> attr_done[kMaxDevices] = {};
     cudaError_t e = setup_once(attr_done, dev, [] {
-        return cudaFuncSetAttribute(wq::smallm_kernel<BITS, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)kSmemMax);
+        cudaError_t r = cudaSuccess;
+        const void *fs[4] = {(const void *)wq::smallm_kernel<BITS, TOK, 1>, (const void *)wq::smallm_kernel<BITS, TOK, 2>,
+                             (const void *)wq::smallm_kernel<BITS, TOK, 3>,
+                             (const void *)wq::smallm_kernel<BITS, TOK, wq::sm_max_rb<TOK>()>};
+        for (const void *f : fs)
+            if (r == cudaSuccess) r = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax);
+        return r;
     });
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smallm)");
     const int64_t U = (a.N + 15) / 16;
@@ -294,7 +327,10 @@ wq_status launch_smallm_tok(wq::SmallMArgs a, int dev, int sm_count, cudaStream_
             smem = total;
         }
     }
-    if (best < 0) return fail(WQ_ERR_INVALID_ARG, "no shared-memory layout for the small-M kernel");
+    if (best < 0) {
+        *no_layout = true;
+        return fail(WQ_ERR_INVALID_ARG, "no shared-memory layout for the small-M kernel");
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(chosen.n_clusters * chosen.S));
     cfg.blockDim = dim3(wq::SmCfg<TOK>::kThreads);
@@ -318,24 +354,44 @@ wq_status launch_smallm_tok(wq::SmallMArgs a, int dev, int sm_count, cudaStream_
     }
     cfg.attrs = attr;
     cfg.numAttrs = n_attr;
-    e = cudaLaunchKernelEx(&cfg, wq::smallm_kernel<BITS, TOK>, chosen);
+    switch (chosen.RB) {
+        case 1: e = smallm_launch_rb<BITS, TOK, 1>(cfg, pm, chosen); break;
+        case 2: e = smallm_launch_rb<BITS, TOK, 2>(cfg, pm, chosen); break;
+        case 3: e = smallm_launch_rb<BITS, TOK, 3>(cfg, pm, chosen); break;
+        default: e = smallm_launch_rb<BITS, TOK, wq::sm_max_rb<TOK>()>(cfg, pm, chosen); break;
+    }
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(smallm_kernel)");
     return check_launch("smallm_kernel");
 }
 
-// Up to 16 tokens per launch; more tokens take several launches.
+// Up to 16 tokens per launch; more tokens take several launches. A shape whose staged x
+// and partial sums do not fit in shared memory for 16 tokens is run in launches of 8, 4, 2
+// or 1 tokens (each streams the weight once more). The packed codes are read by TMA as
+// [N][K*b/8] bytes, one unit (16 rows x 16*b bytes of one group) per copy.
 template <int BITS>
-wq_status launch_smallm(const wq::SmallMArgs &base, int dev, int sm_count, cudaStream_t st) {
-    for (int64_t m0 = 0; m0 < base.M; m0 += wq::kSmMaxTok) {
+wq_status launch_smallm(const wq::SmallMArgs &base, const uint8_t *packed, int dev, int sm_count, cudaStream_t st) {
+    CUtensorMap pm;
+    const uint64_t row_bytes = (uint64_t)base.K * BITS / 8;
+    wq_status s = make_map_2d(&pm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, row_bytes, (uint64_t)base.N, row_bytes,
+                              16u * BITS, 16u, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (s != WQ_OK) return s;
+    int64_t chunk = wq::kSmMaxTok;
+    for (int64_t m0 = 0; m0 < base.M;) {
         wq::SmallMArgs a = base;
-        a.M = std::min<int64_t>(wq::kSmMaxTok, base.M - m0);
+        a.M = std::min<int64_t>(chunk, base.M - m0);
         a.x = base.x + m0 * base.K;
         a.y = base.y + m0 * base.N;
         if (base.t) a.t = base.t + m0 * wq::kTStrideSm;
-        wq_status s;
-        if (a.M <= 8) s = launch_smallm_tok<BITS, 8>(a, dev, sm_count, st);
-        else s = launch_smallm_tok<BITS, 16>(a, dev, sm_count, st);
+        bool no_layout = false;
+        if (a.M <= 8) s = launch_smallm_tok<BITS, 8>(a, pm, dev, sm_count, st, &no_layout);
+        else s = launch_smallm_tok<BITS, 16>(a, pm, dev, sm_count, st, &no_layout);
+        if (no_layout && a.M > 1) {
+            chunk = (a.M + 1) / 2;                     // nothing was launched: retry with fewer tokens
+            g_last_error[0] = 0;
+            continue;
+        }
         if (s != WQ_OK) return s;
+        m0 += a.M;
     }
     return WQ_OK;
 }
@@ -788,8 +844,6 @@ wq_status wq_linear_ex(const void *x, int64_t M, int64_t K, const uint8_t *packe
 
     wq::SmallMArgs a{};
     a.x = static_cast<const uint16_t *>(x);
-    a.packed = packed;
-    a.row_bytes = K * bits / 8;
     a.scales = scales;
     a.bias = static_cast<const uint16_t *>(bias);
     a.L2 = static_cast<const uint16_t *>(L2);
@@ -811,11 +865,11 @@ wq_status wq_linear_ex(const void *x, int64_t M, int64_t K, const uint8_t *packe
         a.t = t;
     }
     switch (bits) {
-        case 3: return launch_smallm<3>(a, dev, info->sm_count, st);
-        case 4: return launch_smallm<4>(a, dev, info->sm_count, st);
-        case 5: return launch_smallm<5>(a, dev, info->sm_count, st);
-        case 6: return launch_smallm<6>(a, dev, info->sm_count, st);
-        default: return launch_smallm<7>(a, dev, info->sm_count, st);
+        case 3: return launch_smallm<3>(a, packed, dev, info->sm_count, st);
+        case 4: return launch_smallm<4>(a, packed, dev, info->sm_count, st);
+        case 5: return launch_smallm<5>(a, packed, dev, info->sm_count, st);
+        case 6: return launch_smallm<6>(a, packed, dev, info->sm_count, st);
+        default: return launch_smallm<7>(a, packed, dev, info->sm_count, st);
     }
 }
 
