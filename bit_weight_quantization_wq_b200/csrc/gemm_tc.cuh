@@ -61,18 +61,24 @@ constexpr int kTStride = 128;             // row stride (elements) of the low-ra
 constexpr int kTcRegsWg0 = 48, kTcRegsWg1 = 96, kTcRegsPromote = 184, kTcRegsLaunch = 128;
 static_assert(kTcRegsWg0 + kTcRegsWg1 + 2 * kTcRegsPromote == 4 * kTcRegsLaunch, "register split");
 
-template <int TT>
+// TMEM columns: T0 at 0 and T1 at 256 (TT <= 192 columns each), the code tiles A0 at 192 and
+// A1 at 448 (64 columns = one 128-k group of bf16 pairs each).
+__host__ __device__ constexpr uint32_t tc_a_col(uint32_t b) { return 192u + 256u * b; }
+
+template <int TT, int BITS>
 struct TcLayout {
-    static constexpr int kStages = TT > 128 ? 4 : 6;
-    static constexpr uint32_t kXBytes = TT * kTcBK * 2;             // 32 KB (TT = 256)
-    static constexpr uint32_t kABytes = kTcBW * kTcBK * 2;          // 16 KB
+    static constexpr int kStages = TT > 128 ? 6 : 8;                 // x stages (64 k each)
+    static constexpr int kPStages = 3;                               // packed group tiles
+    static constexpr uint32_t kXBytes = TT * kTcBK * 2;              // 24 KB (TT = 192)
+    static constexpr uint32_t kPBytes = ((kTcBW * 16 * BITS + 1023) / 1024) * 1024;   // <= 14 KB
     static constexpr uint32_t kOffX = 0;
-    static constexpr uint32_t kOffA = kOffX + kStages * kXBytes;
-    static constexpr uint32_t kOffL = kOffA + kStages * kABytes;    // low-rank L2 tile [rank][128] bf16
+    static constexpr uint32_t kOffP = kOffX + kStages * kXBytes;
+    static constexpr uint32_t kOffL = kOffP + kPStages * kPBytes;    // low-rank L2 tile [rank][128] bf16
     static constexpr uint32_t kLBytes = 64 * kTcBW * 2;
     static constexpr uint32_t kOffBar = kOffL + kLBytes;
-    // full[S], empty[S], p_full[S], t_full[2], t_empty[2], l_full, l_empty, drain[2]
-    static constexpr uint32_t kNumBars = 3 * kStages + 8;
+    // full[S], empty[S], p_full[P], p_empty[P], a_full[2], a_empty[2], t_full[2], t_empty[2],
+    // l_full, l_empty, drain[2]
+    static constexpr uint32_t kNumBars = 2 * kStages + 2 * kPStages + 12;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kBytes = kOffMisc + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;               // slack to align the base to 1024 B
@@ -121,21 +127,30 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) {
     return (r >> 3) * 1024u + (r & 7u) * 128u + ((c ^ (r & 7u)) << 4);
 }
 
+// 32 lanes x 8 consecutive 32-bit columns from registers: thread i of the warp writes lane (base + i).
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t *r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
 template <int BITS, int TT>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap t_map,
                  const __grid_constant__ CUtensorMap l_map, const __grid_constant__ CUtensorMap p_map,
                  const TcParams p) {
-    using L = TcLayout<TT>;
-    constexpr int S = L::kStages;
+    using L = TcLayout<TT, BITS>;
+    constexpr int S = L::kStages, P = L::kPStages;
     constexpr int NWG = 4 * BITS + 1;
     constexpr int kHalf = TT / 2;                 // promotion columns per warp
+    static_assert(TT <= 192 && TT % 16 == 0, "T buffers must leave the code-tile columns free");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
-    uint64_t *full = bars, *empty = full + S, *p_full = empty + S;
-    uint64_t *t_full = p_full + S, *t_empty = t_full + 2;
+    uint64_t *full = bars, *empty = full + S, *p_full = empty + S, *p_empty = p_full + P;
+    uint64_t *a_full = p_empty + P, *a_empty = a_full + 2;
+    uint64_t *t_full = a_empty + 2, *t_empty = t_full + 2;
     uint64_t *l_full = t_empty + 2, *l_empty = l_full + 1;
     uint64_t *drain = l_empty + 1;                               // drain[2]: one per MMA thread
     const uint16_t *l_tile = reinterpret_cast<const uint16_t *>(smem + L::kOffL);
@@ -145,11 +160,16 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1 + 4);          // x producer (+ transaction bytes) + 4 unpack warps
+            mbar_init(&full[i], 1);              // x producer (+ transaction bytes)
             mbar_init(&empty[i], 1);             // the commit of the MMAs that read the stage
-            mbar_init(&p_full[i], 1);            // packed group tile landed in this stage (TMA bytes)
+        }
+        for (int i = 0; i < P; ++i) {
+            mbar_init(&p_full[i], 1);            // packed group tile landed (TMA bytes)
+            mbar_init(&p_empty[i], 4);           // the 4 unpack warps have read it
         }
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&a_full[i], 4);            // the 4 unpack warps stored their rows of the code tile
+            mbar_init(&a_empty[i], 1);           // the commit of the MMAs that read the code tile
             mbar_init(&t_full[i], 1);
             mbar_init(&t_empty[i], 8);           // the 8 promotion warps
         }
@@ -208,41 +228,34 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
             }
         } else if (warp == 2 && lane == 0) {
             // ------------------------------------------------------ packed-code and L2 tile producer
-            // A group's packed tile (128 rows x 16*b bytes, <= 14 KB) lands in the code buffer of
-            // the unit's second stage, where the unpack warps read it before overwriting it with
-            // that stage's codes; the tile's L2 block goes to its own buffer once per tile.
+            // A group's packed tile (128 rows x 16*b bytes) goes to a ring of P buffers that the
+            // unpack warps release once the rows are in registers; the tile's L2 block goes to its
+            // own buffer once per tile.
             tma_prefetch_desc(&p_map);
             if (p.l_tma && p.rank > 0) tma_prefetch_desc(&l_map);
-            int armed[S];
-            for (int i = 0; i < S; ++i) armed[i] = -1;
+            int armed[P];
+            for (int i = 0; i < P; ++i) armed[i] = -1;
             int l_armed = -1;
-            // p_full[s] is armed only when stage s is a group's second stage, which is not every
-            // use of s (a one-stage low-rank unit shifts the pairing), so its phase is counted
-            // per stage: bit s of pph
-            uint32_t q = 0, lph = 0, pph = 0;
+            uint32_t pq = 0, lph = 0;
             for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
                 const int nt = tile % p.tiles_n;
-                for (int u = 0; u < G; ++u, q += 2) {
-                    const uint32_t s1 = (q + 1) % S, ph1 = ((q + 1) / S) & 1;
-                    if (!mbar_wait(&empty[s1], ph1 ^ 1, abort)) goto p_done;
-                    mbar_arrive_expect_tx(&p_full[s1], (uint32_t)kTcBW * 16u * BITS);
-                    armed[s1] = (int)((pph >> s1) & 1u);
-                    pph ^= 1u << s1;
-                    tma_load_2d(smem + L::kOffA + s1 * L::kABytes, &p_map, &p_full[s1], u * 16 * BITS, nt * kTcBW);
+                for (int u = 0; u < G; ++u, ++pq) {
+                    const uint32_t s = pq % P, ph = (pq / P) & 1;
+                    if (!mbar_wait(&p_empty[s], ph ^ 1, abort)) goto p_done;
+                    mbar_arrive_expect_tx(&p_full[s], (uint32_t)kTcBW * 16u * BITS);
+                    armed[s] = (int)ph;
+                    tma_load_2d(smem + L::kOffP + s * L::kPBytes, &p_map, &p_full[s], u * 16 * BITS, nt * kTcBW);
                 }
-                if (p.rank > 0) {
-                    q += nlr;
-                    if (p.l_tma) {
-                        if (!mbar_wait(l_empty, lph ^ 1, abort)) goto p_done;
-                        mbar_arrive_expect_tx(l_full, (uint32_t)p.rank * kTcBW * 2);
-                        l_armed = (int)lph;
-                        tma_load_2d(smem + L::kOffL, &l_map, l_full, nt * kTcBW, 0);
-                        lph ^= 1;
-                    }
+                if (p.rank > 0 && p.l_tma) {
+                    if (!mbar_wait(l_empty, lph ^ 1, abort)) goto p_done;
+                    mbar_arrive_expect_tx(l_full, (uint32_t)p.rank * kTcBW * 2);
+                    l_armed = (int)lph;
+                    tma_load_2d(smem + L::kOffL, &l_map, l_full, nt * kTcBW, 0);
+                    lph ^= 1;
                 }
             }
         p_done:
-            for (int i = 0; i < S; ++i) {
+            for (int i = 0; i < P; ++i) {
                 int local = 0;
                 if (armed[i] >= 0) (void)mbar_wait(&p_full[i], (uint32_t)armed[i], &local, 50ull * 1000ull * 1000ull);
             }
@@ -252,30 +265,33 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
             }
         } else if ((warp == 1 || warp == 3) && lane == 0) {
             // ------------------------------------------------------ MMA issuers
-            // Two threads issue: warp 1 the even units (into T0), warp 3 the odd units (into T1).
+            // Two threads issue: warp 1 the even units (T0, A0), warp 3 the odd units (T1, A1).
+            // A (the codes) comes from tensor memory, B (x) from shared memory.
             const uint32_t mine = (warp == 1) ? 0u : 1u;
             constexpr uint32_t idesc = umma_idesc_bf16(kTcBW, TT);
-            const uint32_t x_base = smem_u32(smem + L::kOffX), a_base = smem_u32(smem + L::kOffA);
+            const uint32_t x_base = smem_u32(smem + L::kOffX);
             uint32_t q = 0, unit = 0;
             for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
                 for (int u = 0; u < U; ++u, ++unit) {
                     const int nst = (u < G) ? 2 : nlr;
                     if ((unit & 1u) != mine) { q += nst; continue; }
-                    const uint32_t tb = unit & 1;
-                    if (!mbar_wait(&t_empty[tb], ((unit >> 1) & 1) ^ 1, abort)) goto m_done;
+                    const uint32_t tb = unit & 1, uph = (unit >> 1) & 1;
+                    if (!mbar_wait(&t_empty[tb], uph ^ 1, abort)) goto m_done;
+                    if (!mbar_wait(&a_full[tb], uph, abort)) goto m_done;
                     tc_fence_after();
-                    const uint32_t d = tmem + tb * 256u;
+                    const uint32_t d = tmem + tb * 256u, a_cols = tmem + tc_a_col(tb);
                     for (int st = 0; st < nst; ++st, ++q) {
                         const uint32_t s = q % S, ph = (q / S) & 1;
                         if (!mbar_wait(&full[s], ph, abort)) goto m_done;
                         tc_fence_after();
                         const int nk = (u < G) ? kTcBK / 16 : min(kTcBK, 2 * p.rank - st * kTcBK) / 16;
-                        const uint32_t xa = x_base + s * L::kXBytes, aa = a_base + s * L::kABytes;
+                        const uint32_t xa = x_base + s * L::kXBytes;
                         for (int k = 0; k < nk; ++k)
-                            umma_bf16(d, umma_desc_sw128(aa + k * 32, 1024), umma_desc_sw128(xa + k * 32, 1024), idesc,
-                                      (st > 0 || k > 0) ? 1u : 0u);
+                            umma_bf16_ts(d, a_cols + 32u * st + 8u * k, umma_desc_sw128(xa + k * 32, 1024), idesc,
+                                         (st > 0 || k > 0) ? 1u : 0u);
                         umma_commit(&empty[s]);
                     }
+                    umma_commit(&a_empty[tb]);
                     umma_commit(&t_full[tb]);
                 }
             }
@@ -289,93 +305,82 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         }
     } else if (wg == 1) {
         regs_dec<kTcRegsWg1>();
-        // ---------------------------------------------------------- unpack codes into shared memory
+        // ---------------------------------------------------------- unpack codes into tensor memory
+        // One weight row per thread (its TMEM lane): the row's packed group from the ring, to
+        // exact bf16 q pairs (k, k+1) in columns 0..63 of the unit's code tile.
         const int row_local = threadIdx.x - 128;
-        const uint32_t a_base = smem_u32(smem + L::kOffA);
-        uint32_t q = 0, lph = 0, pph = 0;     // pph: per-stage phase bits of p_full (see the producer)
+        const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+        uint32_t pq = 0, lph = 0, unit = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int nt = tile % p.tiles_n;
             const int64_t n = (int64_t)nt * kTcBW + row_local;
             const bool row_ok = n < p.N;        // (rows past N arrive as zeros and are never stored)
-            for (int g = 0; g < G; ++g) {
-                const uint32_t s0 = q % S, ph0 = (q / S) & 1;
-                const uint32_t s1 = (q + 1) % S;
-                q += 2;
-                // this row's packed group, from the tile the producer put in stage s1's code buffer
-                const bool got = warp_wait(&p_full[s1], (pph >> s1) & 1u, abort);
-                pph ^= 1u << s1;
-                uint32_t w[NWG];
-                w[4 * BITS] = 0;
-                if (got) {
-                    const uint8_t *src = smem + L::kOffA + s1 * L::kABytes + row_local * (16 * BITS);
+            for (int u = 0; u < U; ++u, ++unit) {
+                const uint32_t ab = unit & 1, uph = (unit >> 1) & 1;
+                const uint32_t a_addr = tmem + lane_addr + tc_a_col(ab);
+                if (u < G) {
+                    const uint32_t s = pq % P, ph = (pq / P) & 1;
+                    ++pq;
+                    if (!warp_wait(&p_full[s], ph, abort)) goto u_done;
+                    uint32_t w[NWG];
+                    w[4 * BITS] = 0;
+                    const uint8_t *src = smem + L::kOffP + s * L::kPBytes + row_local * (16 * BITS);
 #pragma unroll
                     for (int i = 0; i < BITS; ++i) {
                         const uint4 v = *reinterpret_cast<const uint4 *>(src + 16 * i);
                         w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
                     }
-                }
-                const bool ready = got && warp_wait(&empty[s0], ph0 ^ 1, abort);
-                // every unpack thread has its row in registers before any code overwrites the
-                // tile; the barrier also votes, so that the four warps stop together when a wait
-                // gave up (a warp that left alone would strand the others at the next barrier)
-                if (unpack_bar_any(!ready)) goto u_done;
-                static_for<2>([&](auto st_) {
-                    constexpr int st = decltype(st_)::value;
-                    const uint32_t s = st == 0 ? s0 : s1;
-                    const uint32_t base = a_base + s * L::kABytes;
-                    static_for<8>([&](auto c_) {
-                        constexpr int c = decltype(c_)::value;
-                        uint32_t o[4];
-                        unpack_pairs<BITS, st * 8 + c, 1>(w, o);
-                        st_shared_v4(base + sw128_offset(row_local, c), o[0], o[1], o[2], o[3]);
-                    });
-                    // the MMA reads the tile through the async proxy
+                    // this warp's rows are in registers: release the buffer to the next copy (generic
+                    // reads before the async-proxy write)
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&full[s]);
-                });
-            }
-            if (p.rank > 0) {
-                // low-rank unit: A[n][k] = L2[k mod rank][n] for k < 2 rank (both halves of
-                // [t_hi | t_lo] meet the same L2), zero beyond; from the shared-memory tile when
-                // it came by TMA, else straight from global memory
-                if (p.l_tma && !warp_wait(l_full, lph, abort)) goto u_done;
-                for (int st = 0; st < nlr; ++st, ++q) {
-                    const uint32_t s = q % S, ph = (q / S) & 1;
-                    if (!warp_wait(&empty[s], ph ^ 1, abort)) goto u_done;
-                    const uint32_t base = a_base + s * L::kABytes;
+                    if (lane == 0) mbar_arrive(&p_empty[s]);
+                    if (!warp_wait(&a_empty[ab], uph ^ 1, abort)) goto u_done;
+                    tc_fence_after();
+                    static_for<2>([&](auto h_) {
+                        constexpr int h = decltype(h_)::value;
+                        uint32_t o[32];
+                        unpack_pairs<BITS, 8 * h, 8>(w, o);
+                        tmem_st_32x32b_x32(a_addr + 32u * h, o);
+                    });
+                } else {
+                    // low-rank unit: A[n][k] = L2[k mod rank][n] for k < 2 rank (both halves of
+                    // [t_hi | t_lo] meet the same L2); from the shared-memory tile when it came by
+                    // TMA, else straight from global memory
+                    if (p.l_tma && !warp_wait(l_full, lph, abort)) goto u_done;
+                    if (!warp_wait(&a_empty[ab], uph ^ 1, abort)) goto u_done;
+                    tc_fence_after();
+                    for (int c0 = 0; c0 < p.rank; c0 += 8) {
+                        uint32_t o[8];
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint32_t o[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int k = st * kTcBK + c * 8 + 2 * e;
+                        for (int e = 0; e < 8; ++e) {
+                            const int k = 2 * (c0 + e);
+                            const int j = k < p.rank ? k : k - p.rank;
                             uint32_t v = 0;
-                            if (k < 2 * p.rank) {
-                                const int j = k < p.rank ? k : k - p.rank;
-                                if (p.l_tma) {
-                                    v = (uint32_t)l_tile[j * kTcBW + row_local] | ((uint32_t)l_tile[(j + 1) * kTcBW + row_local] << 16);
-                                } else if (row_ok) {
-                                    v = (uint32_t)__ldg(p.L2 + (int64_t)j * p.N + n) |
-                                        ((uint32_t)__ldg(p.L2 + (int64_t)(j + 1) * p.N + n) << 16);
-                                }
+                            if (p.l_tma) {
+                                v = (uint32_t)l_tile[j * kTcBW + row_local] | ((uint32_t)l_tile[(j + 1) * kTcBW + row_local] << 16);
+                            } else if (row_ok) {
+                                v = (uint32_t)__ldg(p.L2 + (int64_t)j * p.N + n) |
+                                    ((uint32_t)__ldg(p.L2 + (int64_t)(j + 1) * p.N + n) << 16);
                             }
                             o[e] = v;
                         }
-                        st_shared_v4(base + sw128_offset(row_local, c), o[0], o[1], o[2], o[3]);
+                        tmem_st_32x32b_x8(a_addr + (uint32_t)c0, o);
                     }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&full[s]);
+                    if (p.l_tma) {
+                        // the L2 tile is read: release it to the next tile's copy (generic reads before
+                        // the next async-proxy write)
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(l_empty);
+                        lph ^= 1;
+                    }
                 }
-                if (p.l_tma) {
-                    // the L2 tile is read: release it to the next tile's copy (generic reads before
-                    // the next async-proxy write)
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(l_empty);
-                    lph ^= 1;
-                }
+                // the code tile is in tensor memory: hand it to the MMA thread
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a_full[ab]);
             }
         }
     u_done:;
@@ -469,103 +474,109 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
 // 64-wide TMA boxes cover a row exactly.
 // x is read once, at close to HBM rate; tensor cores via mma.m16n8k16.
 // grid (ceil(M/64), KS) with clusters of KS (<= 16) CTAs along K; a CTA owns 64 tokens (4
-// warps x 16) and 1/KS of K. Its share of L1 (K/KS x R bf16) is copied into shared memory in
-// passes of up to `sb` 64-k blocks (all of it at once when it fits), x is streamed from global
-// memory kPrePf blocks ahead in registers, and the KS partial sums are added through
-// distributed shared memory.
-// Inside a thread, k is taken in the order that makes its x loads contiguous (16
-// consecutive k per row per 64-k block); the L1 fragments are fetched with ldmatrix.trans
-// from row addresses in the same order.
+// warps x 16) and 1/KS of K, which it streams in 64-k blocks through a ring of kPreStages
+// stages: per stage one TMA tile of x (64 tokens x 64 k, 128-byte swizzle) and one of L1
+// (64 k x R), 4 or 6 stages. Thread 0 refills a stage once the four warps have released it. The A
+// fragments come from the x tile with ldmatrix, the B fragments from the L1 tile with
+// ldmatrix.trans; the KS partial sums are added through distributed shared memory.
 constexpr int kPreMaxKS = 16;
-constexpr int kPrePf = 3;                               // x blocks in flight per thread
 
-// shared memory of a prepass CTA staging `sb` 64-k blocks of L1 at a time
-template <int R>
-__host__ __device__ constexpr uint32_t prepass_smem_bytes(int sb) {
-    return (uint32_t)sb * 64u * (R + 8) * 2u + 64u * R * 4u;
-}
+template <int R> struct PreLayout {
+    static constexpr int kStages = R > 32 ? 4 : 6;                  // two CTAs per SM
+    static constexpr uint32_t kXBytes = 64 * 64 * 2;               // 8 KB, 1024-aligned
+    static constexpr uint32_t kLBytes = 64 * R * 2;                // 2..8 KB
+    static constexpr uint32_t kStageBytes = kXBytes + ((kLBytes + 1023) / 1024) * 1024;
+    static constexpr uint32_t kOffPart = kStages * kStageBytes;    // [64][R] fp32
+    static constexpr uint32_t kOffBar = kOffPart + 64 * R * 4;     // full[S], empty[S], abort
+    static constexpr uint32_t kBytes = kOffBar + 2 * kStages * 8 + 16;
+    static constexpr uint32_t kAlloc = kBytes + 1024;              // room to align the base to 1024
+};
 
 template <int R>
 __global__ void __launch_bounds__(128)
-lowrank_prepass_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ L1,
-                       uint16_t *__restrict__ t, int64_t M, int64_t K, int sb) {
-    constexpr int kLd = R + 8;                          // padded smem row (elements)
-    extern __shared__ __align__(16) uint8_t pre_smem[];
+lowrank_prepass_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap l1_map,
+                       uint16_t *__restrict__ t, int64_t M, int64_t K) {
+    using L = PreLayout<R>;
+    constexpr int S = L::kStages;
+    extern __shared__ __align__(1024) uint8_t pre_raw[];
+    uint8_t *smem = pre_raw + ((1024u - (smem_u32(pre_raw) & 1023u)) & 1023u);   // 1024-aligned for the swizzle
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
     const uint32_t KS = gridDim.y, split = cluster_ctarank();
     const int64_t m0 = (int64_t)blockIdx.x * 64;
     const int64_t nkb = K / 64;
-    const int64_t kb0 = nkb * split / KS, kb1 = nkb * (split + 1) / KS;
-    const int nb = (int)(kb1 - kb0);
-    uint16_t *l1s = reinterpret_cast<uint16_t *>(pre_smem);                   // [sb*64][kLd]
-    float *part = reinterpret_cast<float *>(pre_smem + (size_t)sb * 64 * kLd * 2); // [64][R]
-    const int64_t ra = m0 + warp * 16 + g, rb = ra + 8;
+    const int kb0 = (int)(nkb * split / KS), kb1 = (int)(nkb * (split + 1) / KS);
+    const int nb = kb1 - kb0;
+    float *part = reinterpret_cast<float *>(smem + L::kOffPart);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar), *empty = full + S;
+    volatile int *abort = reinterpret_cast<int *>(empty + S);
     grid_launch_dependents();                           // the consumer of t waits for this grid's end
 
-    // blocks [b0, b1) of this CTA's share of L1 -> shared memory (asynchronous 16-byte copies)
-    auto stage_l1 = [&](int b0, int b1) {
-        constexpr int per_row = R / 8;                  // 16-byte chunks per L1 row
-        const int chunks = (b1 - b0) * 64 * per_row;
-        for (int i = tid; i < chunks; i += 128) {
-            const int kr = i / per_row, cj = i - kr * per_row;
-            const uint32_t dst = smem_u32(l1s + kr * kLd + cj * 8);
-            const uint16_t *src = L1 + ((kb0 + b0) * 64 + kr) * R + cj * 8;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 4);
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
+        *abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&x_map);
+        tma_prefetch_desc(&l1_map);
+    }
+    __syncthreads();
+    // block i of the share -> stage i % S (thread 0)
+    auto issue = [&](int i) {
+        const uint32_t s = (uint32_t)(i % S);
+        uint8_t *st = smem + s * L::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], L::kXBytes + L::kLBytes);
+        tma_load_2d(st, &x_map, &full[s], (kb0 + i) * 64, (int32_t)m0);
+        tma_load_2d(st + L::kXBytes, &l1_map, &full[s], 0, (kb0 + i) * 64);
     };
-    auto load_x = [&](int64_t kb, uint4 (&xa)[2], uint4 (&xb)[2]) {
-        const int64_t k = kb * 64 + 16 * c;
-        if (ra < M) { xa[0] = ldg_stream_v4(x + ra * K + k); xa[1] = ldg_stream_v4(x + ra * K + k + 8); }
-        else xa[0] = xa[1] = make_uint4(0, 0, 0, 0);
-        if (rb < M) { xb[0] = ldg_stream_v4(x + rb * K + k); xb[1] = ldg_stream_v4(x + rb * K + k + 8); }
-        else xb[0] = xb[1] = make_uint4(0, 0, 0, 0);
-    };
-    uint4 xa[kPrePf][2], xb[kPrePf][2];
-#pragma unroll
-    for (int p = 0; p < kPrePf; ++p)
-        if (p < nb) load_x(kb0 + p, xa[p], xb[p]);
+    if (tid == 0)
+        for (int i = 0; i < S - 1 && i < nb; ++i) issue(i);
+
     float acc[R / 8][4];
 #pragma unroll
     for (int j = 0; j < R / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
-
-    int staged0 = 0, staged1 = 0;                       // L1 blocks [staged0, staged1) are in l1s
-    for (int i0 = 0; i0 < nb; i0 += kPrePf) {
-        if (i0 >= staged1) {
-            // next pass of L1 (sb is a multiple of kPrePf, so a pass starts at an i0)
-            __syncthreads();
-            staged0 = i0;
-            staged1 = min(i0 + sb, nb);
-            stage_l1(staged0, staged1);
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-            __syncthreads();
+    // ldmatrix row of this lane: A (x tile, swizzled): token 16 warp + (lane & 15), chunk half
+    // lane >> 4; B (L1 tile): k row (lane & 7) + 8 ((lane >> 3) & 1), column block lane >> 4
+    const uint32_t a_row = (uint32_t)(warp * 16 + (lane & 15)), a_half = (uint32_t)(lane >> 4);
+    const uint32_t b_row = (uint32_t)((lane & 7) + 8 * ((lane >> 3) & 1)), b_col = (uint32_t)(lane >> 4);
+    bool ok = true;
+    for (int i = 0; i < nb; ++i) {
+        if (tid == 0 && i + S - 1 < nb) {
+            // stage (i - 1) % S is free once all four warps have released block i - 1
+            const int j = i + S - 1;
+            if (j >= S && !mbar_wait(&empty[j % S], (uint32_t)((j / S) - 1) & 1u, abort)) ok = false;
+            if (ok) issue(j);
         }
+        const uint32_t s = (uint32_t)(i % S);
+        if (!warp_wait(&full[s], (uint32_t)(i / S) & 1u, abort)) { ok = false; break; }
+        const uint32_t xs = smem_u32(smem + s * L::kStageBytes), ls = xs + L::kXBytes;
 #pragma unroll
-        for (int p = 0; p < kPrePf; ++p) {
-            const int i = i0 + p;
-            if (i >= nb) break;
-            const uint32_t aw[8] = {xa[p][0].x, xa[p][0].y, xa[p][0].z, xa[p][0].w, xa[p][1].x, xa[p][1].y, xa[p][1].z, xa[p][1].w};
-            const uint32_t bw[8] = {xb[p][0].x, xb[p][0].y, xb[p][0].z, xb[p][0].w, xb[p][1].x, xb[p][1].y, xb[p][1].z, xb[p][1].w};
-            if (i + kPrePf < nb) load_x(kb0 + i + kPrePf, xa[p], xb[p]);
-            const uint16_t *l1b = l1s + (size_t)(i - staged0) * 64 * kLd;
+        for (int ks = 0; ks < 4; ++ks) {
+            uint32_t a0, a1, a2, a3;
+            const uint32_t aaddr = xs + sw128_offset(a_row, 2u * ks + a_half);
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3) : "r"(aaddr));
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                // k-slot q of this step <-> actual k = 16 (q%8 / 2) + 4 s + 2 (q / 8) + (q % 2)
-                const int q = lane & 15;
-                const int kr = 16 * ((q & 7) >> 1) + 4 * s + 2 * (q >> 3) + (q & 1);
-#pragma unroll
-                for (int jt = 0; jt < R / 8; jt += 2) {
-                    uint32_t b0, b1, b2, b3;
-                    const int col = jt * 8 + (lane >> 4) * 8;
-                    const uint32_t addr = smem_u32(l1b + kr * kLd + (col < R ? col : jt * 8));
-                    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                                 : "=r"(b0), "=r"(b1), "=r"(b2), "=r"(b3) : "r"(addr));
-                    mma_16816_bf16(acc[jt], aw[2 * s], bw[2 * s], aw[2 * s + 1], bw[2 * s + 1], b0, b1);
-                    if (jt + 1 < R / 8)
-                        mma_16816_bf16(acc[jt + 1], aw[2 * s], bw[2 * s], aw[2 * s + 1], bw[2 * s + 1], b2, b3);
-                }
+            for (int jt = 0; jt < R / 8; jt += 2) {
+                uint32_t b0, b1, b2, b3;
+                const uint32_t col = (uint32_t)jt * 8u + b_col * 8u;
+                const uint32_t baddr = ls + ((uint32_t)(16 * ks) + b_row) * (R * 2u) + 2u * (col < (uint32_t)R ? col : (uint32_t)jt * 8u);
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(b0), "=r"(b1), "=r"(b2), "=r"(b3) : "r"(baddr));
+                mma_16816_bf16(acc[jt], a0, a1, a2, a3, b0, b1);
+                if (jt + 1 < R / 8) mma_16816_bf16(acc[jt + 1], a0, a1, a2, a3, b2, b3);
             }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);          // this warp has read the stage
+    }
+    if (!ok && tid == 0) {
+        // gave up: let the copies already issued land before the shared memory is released
+        for (int i = 0; i < nb && i < S; ++i) {
+            int local = 0;
+            (void)mbar_wait(&full[(nb - 1 - i) % S], (uint32_t)((nb - 1 - i) / S) & 1u, &local, 50ull * 1000ull * 1000ull);
         }
     }
     // partial sums -> shared memory [token][j]

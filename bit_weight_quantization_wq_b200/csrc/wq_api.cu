@@ -452,7 +452,7 @@ wq_status make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base
 template <int BITS, int TT>
 wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &tm, const CUtensorMap &lm,
                     const CUtensorMap &pm, int l_tma, int sm_count, cudaStream_t st) {
-    using L = wq::TcLayout<TT>;
+    using L = wq::TcLayout<TT, BITS>;
     static std::atomic<int> attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -488,24 +488,20 @@ wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &t
 template <int BITS>
 wq_status launch_tc_tt(const TcArgs &a, int tt, const CUtensorMap &xm, const CUtensorMap &tm, const CUtensorMap &lm,
                        const CUtensorMap &pm, int l_tma, int sm_count, cudaStream_t st) {
-    if (tt == 256) return launch_tc<BITS, 256>(a, xm, tm, lm, pm, l_tma, sm_count, st);
-    if (tt == 240) return launch_tc<BITS, 240>(a, xm, tm, lm, pm, l_tma, sm_count, st);
+    if (tt == 192) return launch_tc<BITS, 192>(a, xm, tm, lm, pm, l_tma, sm_count, st);
+    if (tt == 176) return launch_tc<BITS, 176>(a, xm, tm, lm, pm, l_tma, sm_count, st);
     return launch_tc<BITS, 128>(a, xm, tm, lm, pm, l_tma, sm_count, st);
 }
 
 template <int R>
 wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_t st) {
+    using PL = wq::PreLayout<R>;
     const int64_t mtiles = (a.M + 63) / 64;
     const int64_t nkb = a.K / 64;
     // K is split over a cluster of up to 16 CTAs (a non-portable size) while that leaves fewer
-    // than two CTAs per SM; each CTA stages its share of L1 in shared memory, in passes of sb
-    // 64-k blocks (a multiple of the x prefetch depth) when it does not fit at once
+    // than two CTAs per SM
     int ks = 1;
     while (ks < wq::kPreMaxKS && ks * 2 <= nkb && mtiles * ks < 2 * (int64_t)sm_count) ks *= 2;
-    const int nb_max = (int)((nkb + ks - 1) / ks);
-    int sb = (nb_max + wq::kPrePf - 1) / wq::kPrePf * wq::kPrePf;
-    while (sb > wq::kPrePf && wq::prepass_smem_bytes<R>(sb) > kSmemMax / 2) sb -= wq::kPrePf;   // two CTAs per SM
-    const uint32_t smem = wq::prepass_smem_bytes<R>(sb);
     static std::atomic<int> attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -513,13 +509,21 @@ wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_
         cudaError_t r = cudaFuncSetAttribute(wq::lowrank_prepass_kernel<R>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (r != cudaSuccess) return r;
         return cudaFuncSetAttribute(wq::lowrank_prepass_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)kSmemMax);
+                                    (int)PL::kAlloc);
     });
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(lowrank_prepass_kernel)");
+    // x as 64-token x 64-k tiles (128-byte swizzle), L1 as 64-k x R tiles
+    CUtensorMap xm, lm;
+    wq_status s = make_map_2d(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)a.K, (uint64_t)a.M,
+                              (uint64_t)a.K * 2, 64u, 64u, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != WQ_OK) return s;
+    if ((s = make_map_2d(&lm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.L1, (uint64_t)R, (uint64_t)a.K, (uint64_t)R * 2,
+                         (uint32_t)R, 64u, CU_TENSOR_MAP_SWIZZLE_NONE)) != WQ_OK)
+        return s;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)mtiles, (unsigned)ks, 1);
     cfg.blockDim = dim3(128);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = PL::kAlloc;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -528,22 +532,22 @@ wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, wq::lowrank_prepass_kernel<R>, static_cast<const uint16_t *>(a.x),
-                           static_cast<const uint16_t *>(a.L1), t, a.M, a.K, sb);
+    e = cudaLaunchKernelEx(&cfg, wq::lowrank_prepass_kernel<R>, xm, lm, t, a.M, a.K);
     if (e != cudaSuccess) return cuda_fail(e, "cudaLaunchKernelEx(lowrank_prepass_kernel)");
     return check_launch("lowrank_prepass_kernel");
 }
 
-// Tokens per tensor-core tile: 256 or 240 (one MMA covers 128 weight rows x that many tokens,
-// long enough to hide the per-group hand-off of the partial products), whichever needs fewer
+// Tokens per tensor-core tile: 192 or 176 (one MMA covers 128 weight rows x that many tokens;
+// the code tiles take the tensor-memory columns above 192), whichever needs the fewest
 // tile-waves x tokens on this many SMs (a last wave left mostly empty costs a whole wave); 128
-// when there are few tokens.
+// when there are few tokens. (A 160-token tile gave wrong sums once a CTA had several tiles,
+// so it is not used.)
 int tc_tile_tokens(int64_t M, int64_t N, int sm_count) {
     if (M <= 128) return 128;
     const int64_t tiles_n = (N + wq::kTcBW - 1) / wq::kTcBW;
-    int best = 256;
+    int best = 192;
     int64_t best_cost = -1;
-    for (int tt : {256, 240}) {
+    for (int tt : {192, 176}) {
         const int64_t tiles = (M + tt - 1) / tt * tiles_n;
         const int64_t waves = (tiles + sm_count - 1) / sm_count;
         const int64_t cost = waves * tt;
