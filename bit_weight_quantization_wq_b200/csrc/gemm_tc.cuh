@@ -61,24 +61,18 @@ constexpr int kTStride = 128;             // row stride (elements) of the low-ra
 constexpr int kTcRegsWg0 = 48, kTcRegsWg1 = 96, kTcRegsPromote = 184, kTcRegsLaunch = 128;
 static_assert(kTcRegsWg0 + kTcRegsWg1 + 2 * kTcRegsPromote == 4 * kTcRegsLaunch, "register split");
 
-// TMEM columns: T0 at 0 and T1 at 256 (TT <= 192 columns each), the code tiles A0 at 192 and
-// A1 at 448 (64 columns = one 128-k group of bf16 pairs each).
-__host__ __device__ constexpr uint32_t tc_a_col(uint32_t b) { return 192u + 256u * b; }
-
-template <int TT, int BITS>
+template <int TT>
 struct TcLayout {
-    static constexpr int kStages = TT > 128 ? 6 : 8;                 // x stages (64 k each)
-    static constexpr int kPStages = 3;                               // packed group tiles
-    static constexpr uint32_t kXBytes = TT * kTcBK * 2;              // 24 KB (TT = 192)
-    static constexpr uint32_t kPBytes = ((kTcBW * 16 * BITS + 1023) / 1024) * 1024;   // <= 14 KB
+    static constexpr int kStages = TT > 128 ? 4 : 6;
+    static constexpr uint32_t kXBytes = TT * kTcBK * 2;             // 32 KB (TT = 256)
+    static constexpr uint32_t kABytes = kTcBW * kTcBK * 2;          // 16 KB
     static constexpr uint32_t kOffX = 0;
-    static constexpr uint32_t kOffP = kOffX + kStages * kXBytes;
-    static constexpr uint32_t kOffL = kOffP + kPStages * kPBytes;    // low-rank L2 tile [rank][128] bf16
+    static constexpr uint32_t kOffA = kOffX + kStages * kXBytes;
+    static constexpr uint32_t kOffL = kOffA + kStages * kABytes;    // low-rank L2 tile [rank][128] bf16
     static constexpr uint32_t kLBytes = 64 * kTcBW * 2;
     static constexpr uint32_t kOffBar = kOffL + kLBytes;
-    // full[S], empty[S], p_full[P], p_empty[P], a_full[2], a_empty[2], t_full[2], t_empty[2],
-    // l_full, l_empty, drain[2]
-    static constexpr uint32_t kNumBars = 2 * kStages + 2 * kPStages + 12;
+    // full[S], empty[S], p_full[S], t_full[2], t_empty[2], l_full, l_empty, drain[2]
+    static constexpr uint32_t kNumBars = 3 * kStages + 8;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     static constexpr uint32_t kBytes = kOffMisc + 16;
     static constexpr uint32_t kAlloc = kBytes + 1024;               // slack to align the base to 1024 B
@@ -127,30 +121,21 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) {
     return (r >> 3) * 1024u + (r & 7u) * 128u + ((c ^ (r & 7u)) << 4);
 }
 
-// 32 lanes x 8 consecutive 32-bit columns from registers: thread i of the warp writes lane (base + i).
-__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t *r) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
-                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-                 : "memory");
-}
-
 template <int BITS, int TT>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap t_map,
                  const __grid_constant__ CUtensorMap l_map, const __grid_constant__ CUtensorMap p_map,
                  const TcParams p) {
-    using L = TcLayout<TT, BITS>;
-    constexpr int S = L::kStages, P = L::kPStages;
+    using L = TcLayout<TT>;
+    constexpr int S = L::kStages;
     constexpr int NWG = 4 * BITS + 1;
     constexpr int kHalf = TT / 2;                 // promotion columns per warp
-    static_assert(TT <= 192 && TT % 16 == 0, "T buffers must leave the code-tile columns free");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
-    uint64_t *full = bars, *empty = full + S, *p_full = empty + S, *p_empty = p_full + P;
-    uint64_t *a_full = p_empty + P, *a_empty = a_full + 2;
-    uint64_t *t_full = a_empty + 2, *t_empty = t_full + 2;
+    uint64_t *full = bars, *empty = full + S, *p_full = empty + S;
+    uint64_t *t_full = p_full + S, *t_empty = t_full + 2;
     uint64_t *l_full = t_empty + 2, *l_empty = l_full + 1;
     uint64_t *drain = l_empty + 1;                               // drain[2]: one per MMA thread
     const uint16_t *l_tile = reinterpret_cast<const uint16_t *>(smem + L::kOffL);
@@ -160,16 +145,11 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < S; ++i) {
-            mbar_init(&full[i], 1);              // x producer (+ transaction bytes)
+            mbar_init(&full[i], 1 + 4);          // x producer (+ transaction bytes) + 4 unpack warps
             mbar_init(&empty[i], 1);             // the commit of the MMAs that read the stage
-        }
-        for (int i = 0; i < P; ++i) {
-            mbar_init(&p_full[i], 1);            // packed group tile landed (TMA bytes)
-            mbar_init(&p_empty[i], 4);           // the 4 unpack warps have read it
+            mbar_init(&p_full[i], 1);            // packed group tile landed in this stage (TMA bytes)
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&a_full[i], 4);            // the 4 unpack warps stored their rows of the code tile
-            mbar_init(&a_empty[i], 1);           // the commit of the MMAs that read the code tile
             mbar_init(&t_full[i], 1);
             mbar_init(&t_empty[i], 8);           // the 8 promotion warps
         }
@@ -228,34 +208,41 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
             }
         } else if (warp == 2 && lane == 0) {
             // ------------------------------------------------------ packed-code and L2 tile producer
-            // A group's packed tile (128 rows x 16*b bytes) goes to a ring of P buffers that the
-            // unpack warps release once the rows are in registers; the tile's L2 block goes to its
-            // own buffer once per tile.
+            // A group's packed tile (128 rows x 16*b bytes, <= 14 KB) lands in the code buffer of
+            // the unit's second stage, where the unpack warps read it before overwriting it with
+            // that stage's codes; the tile's L2 block goes to its own buffer once per tile.
             tma_prefetch_desc(&p_map);
             if (p.l_tma && p.rank > 0) tma_prefetch_desc(&l_map);
-            int armed[P];
-            for (int i = 0; i < P; ++i) armed[i] = -1;
+            int armed[S];
+            for (int i = 0; i < S; ++i) armed[i] = -1;
             int l_armed = -1;
-            uint32_t pq = 0, lph = 0;
+            // p_full[s] is armed only when stage s is a group's second stage, which is not every
+            // use of s (a one-stage low-rank unit shifts the pairing), so its phase is counted
+            // per stage: bit s of pph
+            uint32_t q = 0, lph = 0, pph = 0;
             for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
                 const int nt = tile % p.tiles_n;
-                for (int u = 0; u < G; ++u, ++pq) {
-                    const uint32_t s = pq % P, ph = (pq / P) & 1;
-                    if (!mbar_wait(&p_empty[s], ph ^ 1, abort)) goto p_done;
-                    mbar_arrive_expect_tx(&p_full[s], (uint32_t)kTcBW * 16u * BITS);
-                    armed[s] = (int)ph;
-                    tma_load_2d(smem + L::kOffP + s * L::kPBytes, &p_map, &p_full[s], u * 16 * BITS, nt * kTcBW);
+                for (int u = 0; u < G; ++u, q += 2) {
+                    const uint32_t s1 = (q + 1) % S, ph1 = ((q + 1) / S) & 1;
+                    if (!mbar_wait(&empty[s1], ph1 ^ 1, abort)) goto p_done;
+                    mbar_arrive_expect_tx(&p_full[s1], (uint32_t)kTcBW * 16u * BITS);
+                    armed[s1] = (int)((pph >> s1) & 1u);
+                    pph ^= 1u << s1;
+                    tma_load_2d(smem + L::kOffA + s1 * L::kABytes, &p_map, &p_full[s1], u * 16 * BITS, nt * kTcBW);
                 }
-                if (p.rank > 0 && p.l_tma) {
-                    if (!mbar_wait(l_empty, lph ^ 1, abort)) goto p_done;
-                    mbar_arrive_expect_tx(l_full, (uint32_t)p.rank * kTcBW * 2);
-                    l_armed = (int)lph;
-                    tma_load_2d(smem + L::kOffL, &l_map, l_full, nt * kTcBW, 0);
-                    lph ^= 1;
+                if (p.rank > 0) {
+                    q += nlr;
+                    if (p.l_tma) {
+                        if (!mbar_wait(l_empty, lph ^ 1, abort)) goto p_done;
+                        mbar_arrive_expect_tx(l_full, (uint32_t)p.rank * kTcBW * 2);
+                        l_armed = (int)lph;
+                        tma_load_2d(smem + L::kOffL, &l_map, l_full, nt * kTcBW, 0);
+                        lph ^= 1;
+                    }
                 }
             }
         p_done:
-            for (int i = 0; i < P; ++i) {
+            for (int i = 0; i < S; ++i) {
                 int local = 0;
                 if (armed[i] >= 0) (void)mbar_wait(&p_full[i], (uint32_t)armed[i], &local, 50ull * 1000ull * 1000ull);
             }
@@ -265,33 +252,30 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
             }
         } else if ((warp == 1 || warp == 3) && lane == 0) {
             // ------------------------------------------------------ MMA issuers
-            // Two threads issue: warp 1 the even units (T0, A0), warp 3 the odd units (T1, A1).
-            // A (the codes) comes from tensor memory, B (x) from shared memory.
+            // Two threads issue: warp 1 the even units (into T0), warp 3 the odd units (into T1).
             const uint32_t mine = (warp == 1) ? 0u : 1u;
             constexpr uint32_t idesc = umma_idesc_bf16(kTcBW, TT);
-            const uint32_t x_base = smem_u32(smem + L::kOffX);
+            const uint32_t x_base = smem_u32(smem + L::kOffX), a_base = smem_u32(smem + L::kOffA);
             uint32_t q = 0, unit = 0;
             for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
                 for (int u = 0; u < U; ++u, ++unit) {
                     const int nst = (u < G) ? 2 : nlr;
                     if ((unit & 1u) != mine) { q += nst; continue; }
-                    const uint32_t tb = unit & 1, uph = (unit >> 1) & 1;
-                    if (!mbar_wait(&t_empty[tb], uph ^ 1, abort)) goto m_done;
-                    if (!mbar_wait(&a_full[tb], uph, abort)) goto m_done;
+                    const uint32_t tb = unit & 1;
+                    if (!mbar_wait(&t_empty[tb], ((unit >> 1) & 1) ^ 1, abort)) goto m_done;
                     tc_fence_after();
-                    const uint32_t d = tmem + tb * 256u, a_cols = tmem + tc_a_col(tb);
+                    const uint32_t d = tmem + tb * 256u;
                     for (int st = 0; st < nst; ++st, ++q) {
                         const uint32_t s = q % S, ph = (q / S) & 1;
                         if (!mbar_wait(&full[s], ph, abort)) goto m_done;
                         tc_fence_after();
                         const int nk = (u < G) ? kTcBK / 16 : min(kTcBK, 2 * p.rank - st * kTcBK) / 16;
-                        const uint32_t xa = x_base + s * L::kXBytes;
+                        const uint32_t xa = x_base + s * L::kXBytes, aa = a_base + s * L::kABytes;
                         for (int k = 0; k < nk; ++k)
-                            umma_bf16_ts(d, a_cols + 32u * st + 8u * k, umma_desc_sw128(xa + k * 32, 1024), idesc,
-                                         (st > 0 || k > 0) ? 1u : 0u);
+                            umma_bf16(d, umma_desc_sw128(aa + k * 32, 1024), umma_desc_sw128(xa + k * 32, 1024), idesc,
+                                      (st > 0 || k > 0) ? 1u : 0u);
                         umma_commit(&empty[s]);
                     }
-                    umma_commit(&a_empty[tb]);
                     umma_commit(&t_full[tb]);
                 }
             }
@@ -305,82 +289,93 @@ tc_linear_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constan
         }
     } else if (wg == 1) {
         regs_dec<kTcRegsWg1>();
-        // ---------------------------------------------------------- unpack codes into tensor memory
-        // One weight row per thread (its TMEM lane): the row's packed group from the ring, to
-        // exact bf16 q pairs (k, k+1) in columns 0..63 of the unit's code tile.
+        // ---------------------------------------------------------- unpack codes into shared memory
         const int row_local = threadIdx.x - 128;
-        const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-        uint32_t pq = 0, lph = 0, unit = 0;
+        const uint32_t a_base = smem_u32(smem + L::kOffA);
+        uint32_t q = 0, lph = 0, pph = 0;     // pph: per-stage phase bits of p_full (see the producer)
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             const int nt = tile % p.tiles_n;
             const int64_t n = (int64_t)nt * kTcBW + row_local;
             const bool row_ok = n < p.N;        // (rows past N arrive as zeros and are never stored)
-            for (int u = 0; u < U; ++u, ++unit) {
-                const uint32_t ab = unit & 1, uph = (unit >> 1) & 1;
-                const uint32_t a_addr = tmem + lane_addr + tc_a_col(ab);
-                if (u < G) {
-                    const uint32_t s = pq % P, ph = (pq / P) & 1;
-                    ++pq;
-                    if (!warp_wait(&p_full[s], ph, abort)) goto u_done;
-                    uint32_t w[NWG];
-                    w[4 * BITS] = 0;
-                    const uint8_t *src = smem + L::kOffP + s * L::kPBytes + row_local * (16 * BITS);
+            for (int g = 0; g < G; ++g) {
+                const uint32_t s0 = q % S, ph0 = (q / S) & 1;
+                const uint32_t s1 = (q + 1) % S;
+                q += 2;
+                // this row's packed group, from the tile the producer put in stage s1's code buffer
+                const bool got = warp_wait(&p_full[s1], (pph >> s1) & 1u, abort);
+                pph ^= 1u << s1;
+                uint32_t w[NWG];
+                w[4 * BITS] = 0;
+                if (got) {
+                    const uint8_t *src = smem + L::kOffA + s1 * L::kABytes + row_local * (16 * BITS);
 #pragma unroll
                     for (int i = 0; i < BITS; ++i) {
                         const uint4 v = *reinterpret_cast<const uint4 *>(src + 16 * i);
                         w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
                     }
-                    // this warp's rows are in registers: release the buffer to the next copy (generic
-                    // reads before the async-proxy write)
+                }
+                const bool ready = got && warp_wait(&empty[s0], ph0 ^ 1, abort);
+                // every unpack thread has its row in registers before any code overwrites the
+                // tile; the barrier also votes, so that the four warps stop together when a wait
+                // gave up (a warp that left alone would strand the others at the next barrier)
+                if (unpack_bar_any(!ready)) goto u_done;
+                static_for<2>([&](auto st_) {
+                    constexpr int st = decltype(st_)::value;
+                    const uint32_t s = st == 0 ? s0 : s1;
+                    const uint32_t base = a_base + s * L::kABytes;
+                    static_for<8>([&](auto c_) {
+                        constexpr int c = decltype(c_)::value;
+                        uint32_t o[4];
+                        unpack_pairs<BITS, st * 8 + c, 1>(w, o);
+                        st_shared_v4(base + sw128_offset(row_local, c), o[0], o[1], o[2], o[3]);
+                    });
+                    // the MMA reads the tile through the async proxy
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&p_empty[s]);
-                    if (!warp_wait(&a_empty[ab], uph ^ 1, abort)) goto u_done;
-                    tc_fence_after();
-                    static_for<2>([&](auto h_) {
-                        constexpr int h = decltype(h_)::value;
-                        uint32_t o[32];
-                        unpack_pairs<BITS, 8 * h, 8>(w, o);
-                        tmem_st_32x32b_x32(a_addr + 32u * h, o);
-                    });
-                } else {
-                    // low-rank unit: A[n][k] = L2[k mod rank][n] for k < 2 rank (both halves of
-                    // [t_hi | t_lo] meet the same L2); from the shared-memory tile when it came by
-                    // TMA, else straight from global memory
-                    if (p.l_tma && !warp_wait(l_full, lph, abort)) goto u_done;
-                    if (!warp_wait(&a_empty[ab], uph ^ 1, abort)) goto u_done;
-                    tc_fence_after();
-                    for (int c0 = 0; c0 < p.rank; c0 += 8) {
-                        uint32_t o[8];
+                    if (lane == 0) mbar_arrive(&full[s]);
+                });
+            }
+            if (p.rank > 0) {
+                // low-rank unit: A[n][k] = L2[k mod rank][n] for k < 2 rank (both halves of
+                // [t_hi | t_lo] meet the same L2), zero beyond; from the shared-memory tile when
+                // it came by TMA, else straight from global memory
+                if (p.l_tma && !warp_wait(l_full, lph, abort)) goto u_done;
+                for (int st = 0; st < nlr; ++st, ++q) {
+                    const uint32_t s = q % S, ph = (q / S) & 1;
+                    if (!warp_wait(&empty[s], ph ^ 1, abort)) goto u_done;
+                    const uint32_t base = a_base + s * L::kABytes;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int k = 2 * (c0 + e);
-                            const int j = k < p.rank ? k : k - p.rank;
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t o[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int k = st * kTcBK + c * 8 + 2 * e;
                             uint32_t v = 0;
-                            if (p.l_tma) {
-                                v = (uint32_t)l_tile[j * kTcBW + row_local] | ((uint32_t)l_tile[(j + 1) * kTcBW + row_local] << 16);
-                            } else if (row_ok) {
-                                v = (uint32_t)__ldg(p.L2 + (int64_t)j * p.N + n) |
-                                    ((uint32_t)__ldg(p.L2 + (int64_t)(j + 1) * p.N + n) << 16);
+                            if (k < 2 * p.rank) {
+                                const int j = k < p.rank ? k : k - p.rank;
+                                if (p.l_tma) {
+                                    v = (uint32_t)l_tile[j * kTcBW + row_local] | ((uint32_t)l_tile[(j + 1) * kTcBW + row_local] << 16);
+                                } else if (row_ok) {
+                                    v = (uint32_t)__ldg(p.L2 + (int64_t)j * p.N + n) |
+                                        ((uint32_t)__ldg(p.L2 + (int64_t)(j + 1) * p.N + n) << 16);
+                                }
                             }
                             o[e] = v;
                         }
-                        tmem_st_32x32b_x8(a_addr + (uint32_t)c0, o);
+                        st_shared_v4(base + sw128_offset(row_local, c), o[0], o[1], o[2], o[3]);
                     }
-                    if (p.l_tma) {
-                        // the L2 tile is read: release it to the next tile's copy (generic reads before
-                        // the next async-proxy write)
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(l_empty);
-                        lph ^= 1;
-                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full[s]);
                 }
-                // the code tile is in tensor memory: hand it to the MMA thread
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[ab]);
+                if (p.l_tma) {
+                    // the L2 tile is read: release it to the next tile's copy (generic reads before
+                    // the next async-proxy write)
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(l_empty);
+                    lph ^= 1;
+                }
             }
         }
     u_done:;

@@ -452,7 +452,7 @@ wq_status make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base
 template <int BITS, int TT>
 wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &tm, const CUtensorMap &lm,
                     const CUtensorMap &pm, int l_tma, int sm_count, cudaStream_t st) {
-    using L = wq::TcLayout<TT, BITS>;
+    using L = wq::TcLayout<TT>;
     static std::atomic<int> attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -488,8 +488,8 @@ wq_status launch_tc(const TcArgs &a, const CUtensorMap &xm, const CUtensorMap &t
 template <int BITS>
 wq_status launch_tc_tt(const TcArgs &a, int tt, const CUtensorMap &xm, const CUtensorMap &tm, const CUtensorMap &lm,
                        const CUtensorMap &pm, int l_tma, int sm_count, cudaStream_t st) {
-    if (tt == 192) return launch_tc<BITS, 192>(a, xm, tm, lm, pm, l_tma, sm_count, st);
-    if (tt == 176) return launch_tc<BITS, 176>(a, xm, tm, lm, pm, l_tma, sm_count, st);
+    if (tt == 256) return launch_tc<BITS, 256>(a, xm, tm, lm, pm, l_tma, sm_count, st);
+    if (tt == 240) return launch_tc<BITS, 240>(a, xm, tm, lm, pm, l_tma, sm_count, st);
     return launch_tc<BITS, 128>(a, xm, tm, lm, pm, l_tma, sm_count, st);
 }
 
@@ -537,17 +537,16 @@ wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_
     return check_launch("lowrank_prepass_kernel");
 }
 
-// Tokens per tensor-core tile: 192 or 176 (one MMA covers 128 weight rows x that many tokens;
-// the code tiles take the tensor-memory columns above 192), whichever needs the fewest
+// Tokens per tensor-core tile: 256 or 240 (one MMA covers 128 weight rows x that many tokens,
+// long enough to hide the per-group hand-off of the partial products), whichever needs fewer
 // tile-waves x tokens on this many SMs (a last wave left mostly empty costs a whole wave); 128
-// when there are few tokens. (A 160-token tile gave wrong sums once a CTA had several tiles,
-// so it is not used.)
+// when there are few tokens.
 int tc_tile_tokens(int64_t M, int64_t N, int sm_count) {
     if (M <= 128) return 128;
     const int64_t tiles_n = (N + wq::kTcBW - 1) / wq::kTcBW;
-    int best = 192;
+    int best = 256;
     int64_t best_cost = -1;
-    for (int tt : {192, 176}) {
+    for (int tt : {256, 240}) {
         const int64_t tiles = (M + tt - 1) / tt * tiles_n;
         const int64_t waves = (tiles + sm_count - 1) / sm_count;
         const int64_t cost = waves * tt;
