@@ -498,10 +498,11 @@ wq_status launch_prepass(const TcArgs &a, uint16_t *t, int sm_count, cudaStream_
     using PL = wq::PreLayout<R>;
     const int64_t mtiles = (a.M + 63) / 64;
     const int64_t nkb = a.K / 64;
-    // K is split over a cluster of up to 16 CTAs (a non-portable size) while that leaves fewer
-    // than two CTAs per SM
+    // K is split over a cluster of up to 16 CTAs (a non-portable size) while the doubled split
+    // still leaves at most two CTAs per SM (longer CTAs amortize the ring's start and the
+    // cluster reduction)
     int ks = 1;
-    while (ks < wq::kPreMaxKS && ks * 2 <= nkb && mtiles * ks < 2 * (int64_t)sm_count) ks *= 2;
+    while (ks < wq::kPreMaxKS && ks * 2 <= nkb && mtiles * ks * 2 <= 2 * (int64_t)sm_count) ks *= 2;
     static std::atomic<int> attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
