@@ -183,7 +183,10 @@ def run_step(wq, lins, ws, pack, events=None):
 # (prepass + tensor-core kernel, mean over the 3 shapes), recorded from one ncu capture of
 # this workload, keyed by a digest of the kernel sources it was taken on; a changed kernel
 # reports null until it is captured again.
-RECORDED_TRAFFIC = {}
+RECORDED_TRAFFIC = {
+    # 57.0, 131.2 and 248.9 MB for 3072x3072, 12288x3072 and 3072x12288 (N x K)
+    "873ace71abbc1ec1": 145.69e6,
+}
 KERNEL_SOURCES = ("gemm_tc.cuh", "unpack.cuh", "common.cuh", "wq_api.cu")
 
 
