@@ -268,14 +268,11 @@ quantize_pack_many_kernel(const __grid_constant__ PackSegments segs) {
     const int64_t warp_id = (int64_t)blockIdx.x * (kPackThreads / 32) + warp;
     const int64_t n_warps = (int64_t)gridDim.x * (kPackThreads / 32);
     const int64_t v_end = segs.vbegin[segs.n];
+    // the block's segment: a warp's blocks only move forward, so its segment index (the same in
+    // every lane) advances past the segments that end at or before the block
+    int s = 0;
     for (int64_t v0 = warp_id * kPackGroupsPerWarp; v0 < v_end; v0 += n_warps * kPackGroupsPerWarp) {
-        // the block's segment = the number of segments that end at or before v0
-        int s = 0;
-#pragma unroll
-        for (int base = 0; base < kPackMaxSegs; base += 32) {
-            const int j = base + lane;
-            s += __popc(__ballot_sync(0xffffffffu, j < segs.n && segs.vbegin[j + 1] <= v0));
-        }
+        while (s + 1 < segs.n && segs.vbegin[s + 1] <= v0) ++s;
         pack_block<BITS, false>(segs.W[s], segs.n_groups[s], segs.packed[s], segs.scales[s], v0 - segs.vbegin[s],
                                 stage[warp], lane);
     }
